@@ -1,0 +1,163 @@
+"""fp64 CPU oracle for the Ulysses per-rank attention path.
+
+TEST INFRASTRUCTURE ONLY. The tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the library under
+``long_context_sequence_ulysses_b200`` never does, and this package imports
+nothing from it. The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP
+over heads and rows); this module only builds it with gcc and marshals numpy
+arrays through ctypes.
+
+Parity status of each function (what pins it is listed in the tests):
+  seq_to_head, head_to_seq  pinned (hand-derived golden permutation, inverse)
+  doc_start                 pinned (hand-derived golden, definition by brute force)
+  attn_fwd                  pinned (brute force, SDPA, closed forms, invariances)
+  attn_bwd                  pinned (finite differences, autograd, sum rules)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P, I64, I32, F64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
+            lib.oracle_seq_to_head.argtypes = [P, P, I64, I32, I32, I32]
+            lib.oracle_seq_to_head.restype = I32
+            lib.oracle_head_to_seq.argtypes = [P, P, I64, I32, I32, I32]
+            lib.oracle_head_to_seq.restype = I32
+            lib.oracle_doc_start.argtypes = [P, I64, P]
+            lib.oracle_doc_start.restype = None
+            lib.oracle_attn_fwd_rows.argtypes = [P, P, P, P, I64, I32, I32, I32, F64, P, I64, P, P]
+            lib.oracle_attn_fwd_rows.restype = I32
+            lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, I64, I32, I32, I32, F64, P, P, P, P, P]
+            lib.oracle_attn_bwd.restype = I32
+            _lib = lib
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 tensor / uint16 array -> contiguous uint16 numpy array of its bits."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            assert x.dtype == torch.bfloat16, x.dtype
+            return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(x)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def _i32(x) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def seq_to_head(src, N: int, P: int, Hx: int, d: int) -> np.ndarray:
+    """[P][N/P][Hx][d] -> [P][N][Hx/P][d] on raw 16-bit patterns."""
+    s = _bits(src).reshape(-1)
+    dst = np.empty(P * N * (Hx // P) * d if P else 0, dtype=np.uint16)
+    rc = _load().oracle_seq_to_head(_ptr(s), _ptr(dst), N, P, Hx, d)
+    if rc != 0:
+        raise ValueError("oracle_seq_to_head: invalid arguments")
+    return dst.reshape(P, N, Hx // P, d)
+
+
+def head_to_seq(src, N: int, P: int, Hx: int, d: int) -> np.ndarray:
+    """[P][N][Hx/P][d] -> [P][N/P][Hx][d] on raw 16-bit patterns."""
+    s = _bits(src).reshape(-1)
+    dst = np.empty(N * Hx * d, dtype=np.uint16)
+    rc = _load().oracle_head_to_seq(_ptr(s), _ptr(dst), N, P, Hx, d)
+    if rc != 0:
+        raise ValueError("oracle_head_to_seq: invalid arguments")
+    return dst.reshape(P, N // P, Hx, d)
+
+
+def doc_start(pos) -> np.ndarray:
+    p = _i32(pos)
+    out = np.empty(p.shape[0], dtype=np.int32)
+    _load().oracle_doc_start(_ptr(p), p.shape[0], _ptr(out))
+    return out
+
+
+def attn_fwd(q, k, v, pos, scale: Optional[float] = None,
+             rows: Optional[Sequence[int]] = None):
+    """Exact forward attention of one rank's head slice.
+
+    q [N][Hl][d], k/v [N][Hkvl][d] (bf16), pos [N] int.
+    Returns (o, lse): o [N or len(rows)][Hl][d] fp64, lse [Hl][N or len(rows)].
+    ``scale`` defaults to 1/sqrt(d).
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    N, Hl, d = qb.shape
+    Hkvl = kb.shape[1]
+    p = _i32(pos)
+    assert p.shape[0] == N
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    nr = r.shape[0]
+    o = np.empty((Hl, nr, d), dtype=np.float64)
+    lse = np.empty((Hl, nr), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(p), N, Hl, Hkvl, d,
+                                      float(scale), _ptr(r), nr, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd_rows failed ({rc})")
+    return np.ascontiguousarray(o.transpose(1, 0, 2)), lse
+
+
+def attn_bwd(q, k, v, dout, pos, scale: Optional[float] = None):
+    """Exact gradients (dq, dk, dv) of sum(dO * O), plus (o, lse), in fp64."""
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    N, Hl, d = qb.shape
+    Hkvl = kb.shape[1]
+    p = _i32(pos)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq = np.empty((N, Hl, d), dtype=np.float64)
+    dk = np.empty((N, Hkvl, d), dtype=np.float64)
+    dv = np.empty((N, Hkvl, d), dtype=np.float64)
+    o = np.empty((N, Hl, d), dtype=np.float64)
+    lse = np.empty((Hl, N), dtype=np.float64)
+    rc = _load().oracle_attn_bwd(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(p), N, Hl, Hkvl, d,
+                                 float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd failed ({rc})")
+    return dq, dk, dv, o, lse
