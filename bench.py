@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the Ulysses per-rank attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+
+One step = one pass of the whole hot path over the workload, for every
+emulated rank r of P:
+    seq_to_head(Q), seq_to_head(K), seq_to_head(V)   (rank r's head slice)
+    attention forward (doc-bounds scan + tensor-core kernel) -> O, LSE
+    [attention backward when the workload has one]
+    head_to_seq(O)                                     (back to sequence shards)
+The metric is attention TFLOP/s over the step (FLOPs counted over unmasked
+pairs only: 4*d*H*pairs forward, 10*d*H*pairs backward), with the relayout
+GB/s and the dominant kernel's roofline reported beside it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, make_inputs, unmasked_pairs  # noqa: E402
+
+METRIC = "causal packed attn fwd/bwd TFLOP/s + relayout GB/s on 1 B200, % of roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("attn_fwd.cu", "attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh"):
+        p = os.path.join(ROOT, "long_context_sequence_ulysses_b200", "csrc", name)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def lookup_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, valid only while the
+    kernel sources are unchanged since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    sha = kernel_source_sha()
+    for ln in open(TRAFFIC_FILE):
+        ln = ln.strip()
+        if not ln or ln.startswith("#"):
+            continue
+        parts = ln.split()
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[3] == sha:
+            return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def workload_work(w, lengths):
+    pairs = unmasked_pairs(lengths)
+    fwd = 4.0 * w.d * w.H * pairs
+    bwd = 10.0 * w.d * w.H * pairs if w.backward else 0.0
+    elem = 2
+    # relayout bytes (read + write of every element moved): Q, K, V in; O out
+    # (backward adds dO in and dQ, dK, dV out)
+    qkv = (w.N * w.H * w.d + 2 * w.N * w.Hkv * w.d) * elem
+    o = w.N * w.H * w.d * elem
+    relayout = 2 * (qkv + o)
+    if w.backward:
+        relayout += 2 * (o + qkv)
+    return pairs, fwd, bwd, relayout
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import long_context_sequence_ulysses_b200 as U
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = WORKLOADS[args.workload]
+    P = w.P
+    inp = make_inputs(w, device=dev)
+    pos = inp["position_ids"]
+    lengths = inp["lengths"]
+    q_seq, k_seq, v_seq = inp["q"], inp["k"], inp["v"]
+    do_seq = inp.get("do")
+    Hl, Hkvl, d, N = w.Hl, w.Hkvl, w.d, w.N
+    pairs, fwd_flop, bwd_flop, relayout_bytes = workload_work(w, lengths)
+
+    # rank-slice buffers, reused by every emulated rank
+    qs = torch.empty((N, Hl, d), dtype=torch.bfloat16, device=dev)
+    ks = torch.empty((N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    vs = torch.empty((N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    os_ = torch.empty((N, Hl, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((Hl, N), dtype=torch.float32, device=dev)
+    o_seq = torch.empty_like(q_seq)
+    ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
+    if w.backward:
+        dos = torch.empty_like(qs)
+        dqs, dks, dvs = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
+        dq_seq, dk_seq, dv_seq = torch.empty_like(q_seq), torch.empty_like(k_seq), torch.empty_like(v_seq)
+
+    stream = torch.cuda.current_stream(dev)
+    ev = {"attn_fwd": [], "attn_bwd": [], "relayout": []}
+    launches = {"n": 0}
+
+    def timed(kind, fn):
+        if args.kernel_events:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev[kind].append((a, b))
+        else:
+            fn()
+
+    def step(record: bool):
+        for r in range(P):
+            timed("relayout", lambda: U.seq_to_head(q_seq, P, rank=r, out=qs))
+            timed("relayout", lambda: U.seq_to_head(k_seq, P, rank=r, out=ks))
+            timed("relayout", lambda: U.seq_to_head(v_seq, P, rank=r, out=vs))
+            timed("attn_fwd", lambda: U.attn_fwd(qs, ks, vs, pos, out=os_, lse=lse, ws=ws))
+            n = 3 + 4
+            if w.backward:
+                timed("relayout", lambda: U.seq_to_head(do_seq, P, rank=r, out=dos))
+                timed("attn_bwd", lambda: U.attn_bwd(qs, ks, vs, os_, dos, lse, pos, ws=ws, dq=dqs, dk=dks, dv=dvs))
+                timed("relayout", lambda: U.head_to_seq(dqs, P, rank=r, out=dq_seq))
+                timed("relayout", lambda: U.head_to_seq(dks, P, rank=r, out=dk_seq))
+                timed("relayout", lambda: U.head_to_seq(dvs, P, rank=r, out=dv_seq))
+                n += 1 + 8 + 3
+            timed("relayout", lambda: U.head_to_seq(os_, P, rank=r, out=o_seq))
+            n += 1
+            if record:
+                launches["n"] += n
+
+    # warm-up
+    saved = args.kernel_events
+    args.kernel_events = False
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    U.sync_status(ws)
+    args.kernel_events = saved
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    U.sync_status(ws)
+    ms_total = t0.elapsed_time(t1)
+    if dist is not None:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+
+    def avg_ms(kind):
+        xs = [a.elapsed_time(b) for a, b in ev[kind]]
+        return (sum(xs) / len(xs)) if xs else None, (sum(xs) if xs else None)
+
+    fwd_avg, fwd_sum = avg_ms("attn_fwd")
+    bwd_avg, bwd_sum = avg_ms("attn_bwd")
+    rel_avg, rel_sum = avg_ms("relayout")
+
+    total_flop = (fwd_flop + bwd_flop) * world
+    value = total_flop / (ms_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    long_step = ms_total > 1000.0
+    bf16_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+    fwd_flop_launch = fwd_flop / P                     # one launch = one rank's heads
+    achieved = fwd_flop_launch / (fwd_avg * 1e-3) / 1e12 if fwd_avg else None
+    traffic = lookup_traffic("attn_fwd_kernel", w.name)
+
+    # ---- end to end through the public API with host buffers (rank 0 of P only
+    # would understate the copies; the whole job's inputs cross PCIe each step)
+    e2e = run_e2e(U, w, inp, args, dev) if args.e2e_steps > 0 else None
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "N": N, "P": P, "H": w.H, "Hkv": w.Hkv, "d": d, "docs": w.docs,
+            "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
+            "step": "for each of P emulated ranks: seq_to_head(Q,K,V) + attn_fwd" + (" + attn_bwd" if w.backward else "")
+                    + " + head_to_seq(O)",
+            "l2": "inputs larger than L2 (126 MB): Q alone is %d MiB" % (N * w.H * d * 2 >> 20),
+        },
+        "roofline": {
+            "kernel": "attn_fwd_kernel (timed with the doc-bounds scan it is launched with)",
+            "bound": "tensor",
+            "achieved": round(achieved, 2) if achieved else None,
+            "peak": bf16_peak,
+            "peak_source": ("%s %s" % (peak_kind, "sustained" if long_step else "burst")),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / bf16_peak, 4) if achieved else None,
+            "frac_of_spec_2250": round(achieved / SPEC_BF16_TFLOPS, 4) if achieved else None,
+            "traffic": traffic,
+            "flop_per_launch": fwd_flop_launch,
+        },
+        "relayout": {
+            "bytes_per_step": relayout_bytes,
+            "ms_per_step": round(rel_sum / args.steps, 4) if rel_sum else None,
+            "achieved_gbs": round(relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9, 1) if rel_sum else None,
+            "peak_gbs": peaks["hbm_gbs"],
+            "frac": round(relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if rel_sum else None,
+            "frac_of_spec_8000": round(relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9 / SPEC_HBM_GBS, 4) if rel_sum else None,
+        },
+        "attn_fwd_ms_per_launch": round(fwd_avg, 4) if fwd_avg else None,
+        "attn_bwd_ms_per_launch": round(bwd_avg, 4) if bwd_avg else None,
+        "attn_bwd_tflops": round((bwd_flop / P) / (bwd_avg * 1e-3) / 1e12, 2) if bwd_avg else None,
+        "gpu_launches": launches["n"],
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(w, inp, args)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(U, w, inp, args, dev):
+    """Same step through the public API from pinned HOST buffers: each step
+    copies Q, K, V and position ids host->device and reads O and LSE back."""
+    P, N, d = w.P, w.N, w.d
+    hq = inp["q"].cpu().pin_memory()
+    hk = inp["k"].cpu().pin_memory()
+    hv = inp["v"].cpu().pin_memory()
+    hpos = inp["position_ids"].cpu().pin_memory()
+    hdo = inp["do"].cpu().pin_memory() if w.backward else None
+    ho = torch.empty_like(hq).pin_memory()
+    hlse = torch.empty((w.H, N), dtype=torch.float32).pin_memory()
+    dq_, dk_, dv_ = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
+    o_seq = torch.empty_like(inp["q"])
+    lse_all = torch.empty((w.H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ws = torch.empty(U.workspace_bytes(N, w.Hl, w.Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
+    qs = torch.empty((N, w.Hl, d), dtype=torch.bfloat16, device=dev)
+    ks = torch.empty((N, w.Hkvl, d), dtype=torch.bfloat16, device=dev)
+    vs = torch.empty_like(ks)
+    os_ = torch.empty_like(qs)
+    dq_s, dk_s, dv_s, do_s = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(ks), torch.empty_like(qs)
+    gq, gk, gv = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
+    gpos = torch.empty_like(inp["position_ids"])
+    gdo = torch.empty_like(inp["q"]) if w.backward else None
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hpos.numel() * 4 + (hdo.numel() * 2 if w.backward else 0)
+    d2h = ho.numel() * 2 + hlse.numel() * 4 + ((hq.numel() + 2 * hk.numel()) * 2 if w.backward else 0)
+    hdq = torch.empty_like(hq).pin_memory() if w.backward else None
+    hdk = torch.empty_like(hk).pin_memory() if w.backward else None
+    hdv = torch.empty_like(hv).pin_memory() if w.backward else None
+
+    def step():
+        gq.copy_(hq, non_blocking=True)
+        gk.copy_(hk, non_blocking=True)
+        gv.copy_(hv, non_blocking=True)
+        gpos.copy_(hpos, non_blocking=True)
+        if w.backward:
+            gdo.copy_(hdo, non_blocking=True)
+        for r in range(P):
+            U.seq_to_head(gq, P, rank=r, out=qs)
+            U.seq_to_head(gk, P, rank=r, out=ks)
+            U.seq_to_head(gv, P, rank=r, out=vs)
+            U.attn_fwd(qs, ks, vs, gpos, out=os_, lse=lse_all[r * w.Hl:(r + 1) * w.Hl], ws=ws)
+            if w.backward:
+                U.seq_to_head(gdo, P, rank=r, out=do_s)
+                U.attn_bwd(qs, ks, vs, os_, do_s, lse_all[r * w.Hl:(r + 1) * w.Hl], gpos, ws=ws, dq=dq_s, dk=dk_s,
+                           dv=dv_s)
+                U.head_to_seq(dq_s, P, rank=r, out=dq_)
+                U.head_to_seq(dk_s, P, rank=r, out=dk_)
+                U.head_to_seq(dv_s, P, rank=r, out=dv_)
+            U.head_to_seq(os_, P, rank=r, out=o_seq)
+        ho.copy_(o_seq, non_blocking=True)
+        hlse.copy_(lse_all, non_blocking=True)
+        if w.backward:
+            hdq.copy_(dq_, non_blocking=True)
+            hdk.copy_(dk_, non_blocking=True)
+            hdv.copy_(dv_, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.e2e_steps
+    pairs, fwd_flop, bwd_flop, _ = workload_work(w, inp["lengths"])
+    return {"value": round((fwd_flop + bwd_flop) / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": args.e2e_steps}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def _oracle_rows_sample(w, lengths, budget_pairs: float, seed: int):
+    """Rows of rank 0 spread over the sequence, with about `budget_pairs`
+    (query, key) pairs over rank 0's heads in total."""
+    import numpy as np
+    starts = np.cumsum([0] + list(lengths))[:-1]
+    ds = np.repeat(starts, lengths)
+    keys = np.arange(w.N) - ds + 1          # keys per row
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(w.N)
+    cum = np.cumsum(keys[order]) * w.Hl
+    n = int(np.searchsorted(cum, budget_pairs)) + 1
+    rows = np.sort(order[:max(1, min(n, w.N))])
+    return rows, int(keys[rows].sum()) * w.Hl
+
+
+def cpu_baseline(w, inp, args, seconds_target: float = 15.0):
+    """The fp64 oracle timed on this host's cores on a bounded sample of rank
+    0's rows; its rate is scaled to TFLOP/s with the same FLOP count per pair."""
+    import numpy as np
+    import oracle
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    q = inp["q"][:, :w.Hl].contiguous().cpu()
+    k = inp["k"][:, :w.Hkvl].contiguous().cpu()
+    v = inp["v"][:, :w.Hkvl].contiguous().cpu()
+    pos = inp["position_ids"].cpu()
+    # calibrate on a small sample, then size the timed sample to ~seconds_target
+    rows, pr = _oracle_rows_sample(w, inp["lengths"], 2e6, seed=1)
+    t = time.perf_counter()
+    oracle.attn_fwd(q, k, v, pos, rows=rows)
+    dt = max(time.perf_counter() - t, 1e-3)
+    rate = pr / dt
+    rows, pr = _oracle_rows_sample(w, inp["lengths"], rate * seconds_target, seed=2)
+    t = time.perf_counter()
+    oracle.attn_fwd(q, k, v, pos, rows=rows)
+    dt = time.perf_counter() - t
+    flop = 4.0 * w.d * pr
+    return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": "forward attention of %d rows x %d heads of rank 0 (%d query-key pairs, %.1f s)"
+                      % (len(rows), w.Hl, pr, dt)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, device="cpu")
+    steps = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        base = cpu_baseline(w, inp, args, seconds_target=args.ref_seconds)
+        if i >= args.warmup:
+            steps.append(base["value"])
+    value = sum(steps) / len(steps)
+    pairs, fwd_flop, bwd_flop, _ = workload_work(w, inp["lengths"])
+    ms_step = (fwd_flop + bwd_flop) / (value * 1e12) * 1e3
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "N": w.N, "P": w.P, "H": w.H, "Hkv": w.Hkv, "d": w.d, "docs": w.docs,
+                   "note": "each step times the fp64 CPU oracle on a bounded sample of rank 0's rows; "
+                           "ms_per_step is the extrapolated time of the whole step"},
+        "cpu_baseline": dict(base, value=round(value, 6)),
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "b200":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

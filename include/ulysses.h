@@ -1,0 +1,158 @@
+/*
+ * ulysses.h -- C ABI of the Ulysses per-rank attention path on one B200.
+ *
+ * Ulysses sequence parallelism (page "Hugging Face并行加速：10倍提升超长序列训练效率",
+ * section "Ulysses的工作原理"; page "DeepSpeed Ulysses 详解", section
+ * "DeepSpeed-Ulysses 的核心机制") splits a sequence of N tokens over P GPUs,
+ * exchanges the projected Q/K/V with an all-to-all so that every GPU holds the
+ * whole sequence for H/P heads, runs ordinary attention on those heads, and
+ * exchanges the output back to sequence shards. On one GPU the P ranks are
+ * emulated as P buffers and the all-to-all as an in-HBM permutation.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates device memory and keeps no pointer after a call returns.
+ *  - bf16 tensors are contiguous, row-major, 16-byte aligned.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream). Argument errors are detected on the host before any
+ *    launch and return ULYSSES_ERR_INVALID / ULYSSES_ERR_UNSUPPORTED /
+ *    ULYSSES_ERR_WORKSPACE without touching device memory.
+ *  - A launch failure returns ULYSSES_ERR_CUDA.
+ *  - Device-side waits are bounded. A wait that runs out records a flag in
+ *    the workspace and the kernel drains and returns; ulysses_sync_status()
+ *    reports it as ULYSSES_ERR_TIMEOUT. Each attention call clears the flag
+ *    when it starts, so the status describes the latest call on that
+ *    workspace.
+ *  - ulysses_last_error() returns a thread-local message for the last failure.
+ *  - Head dimension d must be 32, 64 or 128.
+ */
+#ifndef ULYSSES_H
+#define ULYSSES_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ULYSSES_OK = 0,
+    ULYSSES_ERR_INVALID = -1,     /* null or misaligned pointer, H % P, Hkv % P, N % P, H % Hkv, d, ... */
+    ULYSSES_ERR_UNSUPPORTED = -2, /* a valid request this build does not implement */
+    ULYSSES_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
+    ULYSSES_ERR_TIMEOUT = -4,     /* a bounded device-side wait ran out */
+    ULYSSES_ERR_WORKSPACE = -5    /* workspace missing or smaller than ulysses_attn_workspace_bytes() */
+} ulysses_status;
+
+/* Thread-local text of the last failure (empty string if none). Never NULL. */
+const char *ulysses_last_error(void);
+
+/* Library version string. */
+const char *ulysses_version(void);
+
+/*
+ * Sequence-to-head exchange (the first all-to-all).
+ * Page "Hugging Face并行加速：10倍提升超长序列训练效率", section "Ulysses的工作原理",
+ * steps 序列分片 and 全体间通信; page "DeepSpeed Ulysses 详解", section
+ * "DeepSpeed-Ulysses 的核心机制", item 3.
+ *
+ *   src  [P][N/P][Hx][d] bf16: rank i's buffer holds tokens [i*N/P, (i+1)*N/P)
+ *        for all Hx heads (this is also the plain [N][Hx][d] layout).
+ *   rank < 0:  dst [P][N][Hx/P][d]: every rank's head slice,
+ *              dst[r][n][h][:] = src[n/(N/P)][n%(N/P)][r*Hx/P + h][:].
+ *   rank = r:  dst [N][Hx/P][d]: rank r's head slice only.
+ * Hx is H for Q and Hkv for K and V. Requires N % P == 0, Hx % P == 0,
+ * d in {32,64,128}; src and dst must not overlap. A bit copy (bit-exact).
+ * N == 0 is a no-op.
+ */
+int ulysses_seq_to_head(const void *src, void *dst, int64_t N, int P, int Hx, int d,
+                        int rank, void *stream);
+
+/*
+ * Head-to-sequence exchange (the second all-to-all), the inverse of
+ * ulysses_seq_to_head. Same page, step 全体间通信复原; page "DeepSpeed Ulysses
+ * 详解", item 5.
+ *
+ *   rank < 0:  src [P][N][Hx/P][d] (every rank's slice) -> dst [P][N/P][Hx][d],
+ *              dst[p][m][r*Hx/P + h][:] = src[r][p*N/P + m][h][:].
+ *   rank = r:  src [N][Hx/P][d] (rank r's slice); writes only heads
+ *              [r*Hx/P, (r+1)*Hx/P) of dst [P][N/P][Hx][d], leaving the rest.
+ */
+int ulysses_head_to_seq(const void *src, void *dst, int64_t N, int P, int Hx, int d,
+                        int rank, void *stream);
+
+/*
+ * Bytes of device workspace that ulysses_attn_fwd (backward = 0) or
+ * ulysses_attn_bwd (backward = 1) need for these sizes. The workspace holds
+ * the per-token document starts, per-tile key ranges, the tile schedule, the
+ * backward's row statistics and a status word. Its contents need not be
+ * initialised by the caller.
+ */
+size_t ulysses_attn_workspace_bytes(int64_t N, int Hl, int Hkvl, int d, int backward);
+
+/*
+ * Attention forward for one rank's head slice ("本地注意力计算": ordinary
+ * attention per head on the full sequence; heads are independent).
+ *
+ *   q     [N][Hl][d]   bf16, query head h uses KV head h / (Hl/Hkvl)
+ *   k, v  [N][Hkvl][d] bf16
+ *   position_ids [N] int32 (device): a document starts wherever the id is 0,
+ *         and at token 0 (page "Ulysses verteilt Millionen-Token-Kontexte auf
+ *         mehrere GPUs", section "Integration in den Hugging-Face-Stack").
+ *   scale softmax scale; <= 0 means 1/sqrt(d).
+ *   o     [N][Hl][d]   bf16 output (round to nearest even).
+ *   lse   [Hl][N]      fp32 natural-log logsumexp of the scaled logits.
+ * Row i attends to keys j with doc_start(i) <= j <= i. Requires Hl % Hkvl == 0.
+ */
+int ulysses_attn_fwd(const void *q, const void *k, const void *v, const int32_t *position_ids,
+                     int64_t N, int Hl, int Hkvl, int d, float scale,
+                     void *o, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Fused form: the same attention, reading rank `rank`'s head slice directly
+ * from the sequence-sharded buffers and writing O straight back to the
+ * sequence-sharded layout, so neither exchange is materialised.
+ *
+ *   q_seq [N][H][d], k_seq / v_seq [N][Hkv][d]  (= [P][N/P][heads][d])
+ *   o_seq [N][H][d]: only heads [rank*H/P, (rank+1)*H/P) are written.
+ *   lse   [H/P][N] for this rank's heads.
+ */
+int ulysses_attn_fwd_fused(const void *q_seq, const void *k_seq, const void *v_seq,
+                           const int32_t *position_ids, int64_t N, int P, int H, int Hkv,
+                           int d, int rank, float scale, void *o_seq, float *lse,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Attention backward for one rank's head slice: gradients of sum(dout * o).
+ *   D_i = sum_c dout_ic o_ic;  P_ij = exp(scale q_i.k_j - lse_i);
+ *   dS_ij = P_ij (dout_i.v_j - D_i);
+ *   dq_i = scale sum_j dS_ij k_j;  dk_j = scale sum_{h in group} sum_i dS_ij q_i;
+ *   dv_j = sum_{h in group} sum_i P_ij dout_i.
+ * Inputs are those of ulysses_attn_fwd plus its outputs o and lse, and the
+ * upstream gradient dout [N][Hl][d]. Outputs dq [N][Hl][d], dk and dv
+ * [N][Hkvl][d], bf16. dq, dk, dv are fully overwritten.
+ */
+int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                     const void *dout, const float *lse, const int32_t *position_ids,
+                     int64_t N, int Hl, int Hkvl, int d, float scale,
+                     void *dq, void *dk, void *dv, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronise `stream` and report the status the latest attention call left
+ * in `ws`: ULYSSES_ERR_TIMEOUT if a bounded device wait ran out, else
+ * ULYSSES_OK (or ULYSSES_ERR_CUDA if synchronisation failed). Clears the flag.
+ */
+int ulysses_sync_status(void *ws, void *stream);
+
+/*
+ * Device-side wait limit in nanoseconds for later launches from this process
+ * (default 1e9). Values <= 0 restore the default.
+ */
+void ulysses_set_wait_limit_ns(int64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ULYSSES_H */

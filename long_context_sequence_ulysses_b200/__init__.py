@@ -1,0 +1,244 @@
+"""Ulysses sequence-parallel attention hot path for one B200 (sm_100a).
+
+Thin ctypes binding over ``libulysses.so`` (declared in ``include/ulysses.h``).
+The functions here only marshal arguments: they check tensor shapes and
+dtypes, allocate outputs and workspace through torch (device memory and
+streams are torch's job), and call the C ABI on the current CUDA stream.
+Every step of the computation runs in the library's CUDA kernels; there is no
+fallback, and importing the package fails if the library has not been built
+(``python -m long_context_sequence_ulysses_b200.build``).
+
+The method (page "Hugging Face并行加速：10倍提升超长序列训练效率", section
+"Ulysses的工作原理"): N tokens are split over P ranks; an all-to-all gives each
+rank the whole sequence for H/P heads; each rank runs attention for its heads;
+a second all-to-all restores sequence sharding. On one GPU the ranks are
+emulated as P buffers and the all-to-alls as in-HBM permutations.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "UlyssesError", "library_path", "seq_to_head", "head_to_seq", "workspace_bytes", "attn_fwd",
+    "attn_fwd_fused", "attn_bwd", "sync_status", "set_wait_limit_ns", "version",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libulysses.so")
+
+ULYSSES_OK = 0
+ULYSSES_ERR_INVALID = -1
+ULYSSES_ERR_UNSUPPORTED = -2
+ULYSSES_ERR_CUDA = -3
+ULYSSES_ERR_TIMEOUT = -4
+ULYSSES_ERR_WORKSPACE = -5
+
+
+class UlyssesError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m long_context_sequence_ulysses_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I64, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    lib.ulysses_last_error.restype = ctypes.c_char_p
+    lib.ulysses_version.restype = ctypes.c_char_p
+    lib.ulysses_seq_to_head.argtypes = [P, P, I64, I32, I32, I32, I32, P]
+    lib.ulysses_head_to_seq.argtypes = [P, P, I64, I32, I32, I32, I32, P]
+    lib.ulysses_attn_workspace_bytes.argtypes = [I64, I32, I32, I32, I32]
+    lib.ulysses_attn_workspace_bytes.restype = SZ
+    lib.ulysses_attn_fwd.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, SZ, P]
+    lib.ulysses_attn_fwd_fused.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, F32, P, P, P, SZ, P]
+    lib.ulysses_attn_bwd.argtypes = [P, P, P, P, P, P, P, I64, I32, I32, I32, F32, P, P, P, P, SZ, P]
+    lib.ulysses_sync_status.argtypes = [P, P]
+    lib.ulysses_set_wait_limit_ns.argtypes = [I64]
+    lib.ulysses_set_wait_limit_ns.restype = None
+    for name in ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_fwd_fused",
+                 "ulysses_attn_bwd", "ulysses_sync_status"):
+        getattr(lib, name).restype = I32
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def version() -> str:
+    return _lib.ulysses_version().decode()
+
+
+def _check(rc: int) -> None:
+    if rc != ULYSSES_OK:
+        raise UlyssesError(rc, _lib.ulysses_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _bf16_cuda(name: str, t: torch.Tensor, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bf16 tensor")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor, got shape {tuple(t.shape)}")
+
+
+def _pos32(pos: torch.Tensor, N: int) -> torch.Tensor:
+    if pos.dim() != 1 or pos.shape[0] != N or not pos.is_cuda:
+        raise ValueError("position_ids must be a 1-D CUDA tensor of length N")
+    if pos.dtype != torch.int32:
+        pos = pos.to(torch.int32)   # argument marshalling: the ABI takes int32 ids
+    return pos.contiguous()
+
+
+def seq_to_head(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """[N][Hx][d] (= P rank buffers [P][N/P][Hx][d]) -> [P][N][Hx/P][d], or
+    rank r's slice [N][Hx/P][d] when ``rank >= 0``."""
+    _bf16_cuda("src", src, 3)
+    N, Hx, d = src.shape
+    shape = (P, N, Hx // P, d) if rank < 0 else (N, Hx // P, d)
+    if out is None:
+        out = torch.empty(shape, dtype=src.dtype, device=src.device)
+    elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != src.dtype:
+        raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
+    _check(_lib.ulysses_seq_to_head(_ptr(src), _ptr(out), N, P, Hx, d, rank, _stream(src)))
+    return out
+
+
+def head_to_seq(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """[P][N][Hx/P][d] -> [N][Hx][d]; with ``rank >= 0`` src is rank r's slice
+    [N][Hx/P][d] and only its heads of ``out`` are written."""
+    if rank < 0:
+        _bf16_cuda("src", src, 4)
+        Pp, N, Hl, d = src.shape
+        if Pp != P:
+            raise ValueError("src.shape[0] must equal P")
+    else:
+        _bf16_cuda("src", src, 3)
+        N, Hl, d = src.shape
+    Hx = Hl * P
+    shape = (N, Hx, d)
+    if out is None:
+        if rank >= 0:
+            raise ValueError("head_to_seq with rank >= 0 needs `out` (other ranks' heads are kept)")
+        out = torch.empty(shape, dtype=src.dtype, device=src.device)
+    elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != src.dtype:
+        raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
+    _check(_lib.ulysses_head_to_seq(_ptr(src), _ptr(out), N, P, Hx, d, rank, _stream(src)))
+    return out
+
+
+def workspace_bytes(N: int, Hl: int, Hkvl: int, d: int, backward: bool = False) -> int:
+    return int(_lib.ulysses_attn_workspace_bytes(N, Hl, Hkvl, d, 1 if backward else 0))
+
+
+def _workspace(ws: Optional[torch.Tensor], nbytes: int, device) -> torch.Tensor:
+    if ws is None or ws.numel() * ws.element_size() < nbytes:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    return ws
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position_ids: torch.Tensor,
+             scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+             lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
+             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Causal document-masked GQA attention of one rank's head slice.
+
+    q [N][Hl][d], k/v [N][Hkvl][d] bf16; position_ids [N]. Returns
+    (o [N][Hl][d] bf16, lse [Hl][N] fp32)."""
+    _bf16_cuda("q", q, 3); _bf16_cuda("k", k, 3); _bf16_cuda("v", v, 3)
+    N, Hl, d = q.shape
+    Hkvl = k.shape[1]
+    if k.shape != (N, Hkvl, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [N][Hkvl][d]")
+    pos = _pos32(position_ids, N)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hl, N), dtype=torch.float32, device=q.device)
+    nbytes = workspace_bytes(N, Hl, Hkvl, d, False)
+    ws = _workspace(ws, nbytes, q.device)
+    sc = 0.0 if scale is None else float(scale)
+    _check(_lib.ulysses_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), N, Hl, Hkvl, d, sc, _ptr(out), _ptr(lse),
+                                 _ptr(ws), ws.numel(), _stream(q)))
+    return out, lse
+
+
+def attn_fwd_fused(q_seq: torch.Tensor, k_seq: torch.Tensor, v_seq: torch.Tensor, position_ids: torch.Tensor,
+                   P: int, rank: int, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                   lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
+                   ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention of rank ``rank``'s heads read straight from the
+    sequence-sharded buffers q_seq [N][H][d], k_seq/v_seq [N][Hkv][d]; O is
+    written into ``out`` [N][H][d] (only this rank's heads)."""
+    _bf16_cuda("q_seq", q_seq, 3); _bf16_cuda("k_seq", k_seq, 3); _bf16_cuda("v_seq", v_seq, 3)
+    N, H, d = q_seq.shape
+    Hkv = k_seq.shape[1]
+    pos = _pos32(position_ids, N)
+    if out is None:
+        out = torch.empty_like(q_seq)
+    Hl, Hkvl = H // P, Hkv // P
+    if lse is None:
+        lse = torch.empty((max(Hl, 1), N), dtype=torch.float32, device=q_seq.device)
+    nbytes = workspace_bytes(N, max(Hl, 1), max(Hkvl, 1), d, False)
+    ws = _workspace(ws, nbytes, q_seq.device)
+    sc = 0.0 if scale is None else float(scale)
+    _check(_lib.ulysses_attn_fwd_fused(_ptr(q_seq), _ptr(k_seq), _ptr(v_seq), _ptr(pos), N, P, H, Hkv, d, rank,
+                                       sc, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q_seq)))
+    return out, lse
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dout: torch.Tensor,
+             lse: torch.Tensor, position_ids: torch.Tensor, scale: Optional[float] = None,
+             ws: Optional[torch.Tensor] = None, dq: Optional[torch.Tensor] = None,
+             dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None
+             ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq, dk, dv) of sum(dout * o) for one rank's head slice."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _bf16_cuda(name, t, 3)
+    N, Hl, d = q.shape
+    Hkvl = k.shape[1]
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (Hl, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [Hl][N] tensor")
+    pos = _pos32(position_ids, N)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = workspace_bytes(N, Hl, Hkvl, d, True)
+    ws = _workspace(ws, nbytes, q.device)
+    sc = 0.0 if scale is None else float(scale)
+    _check(_lib.ulysses_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(pos), N, Hl, Hkvl,
+                                 d, sc, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(q)))
+    return dq, dk, dv
+
+
+def sync_status(ws: torch.Tensor) -> None:
+    """Synchronise the current stream; raise UlyssesError(ULYSSES_ERR_TIMEOUT)
+    if a bounded device-side wait of the last call that used ``ws`` ran out."""
+    _check(_lib.ulysses_sync_status(_ptr(ws), _stream(ws)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _lib.ulysses_set_wait_limit_ns(int(ns))
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

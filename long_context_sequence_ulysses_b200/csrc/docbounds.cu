@@ -1,0 +1,180 @@
+// docbounds.cu -- per-token document starts and per-tile key ranges from
+// position_ids, plus the longest-first tile schedule.
+//
+// Packed documents are masked through position ids rather than a 4-D mask
+// (page "Ulysses verteilt Millionen-Token-Kontexte auf mehrere GPUs", section
+// "Integration in den Hugging-Face-Stack"): a document starts wherever the id
+// is 0 (and at token 0), so
+//     doc_start[i] = max{ j <= i : pos[j] == 0 }   (0 if there is none),
+// an inclusive max-scan of (pos[j] == 0 ? j : 0). Row i attends to keys
+// [doc_start[i], i]; since doc_start never decreases, a 128-row query tile
+// starting at r0 needs key tiles doc_start[r0]/128 .. r0/128 and nothing else.
+//
+// Kernels: a block-local scan, a fix-up with the carry of earlier blocks
+// (which also writes each query tile's first key), for the backward the last
+// query row of each key tile (a binary search over doc_start), and a counting
+// sort of tiles by work, heaviest first.
+#include "ulysses_internal.cuh"
+
+namespace uly {
+
+namespace {
+
+__device__ __forceinline__ int warp_incl_max(int v)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if ((threadIdx.x & 31) >= o) v = max(v, u);
+    }
+    return v;
+}
+
+// Block-local inclusive max-scan over kScanBlock tokens (one per thread).
+__global__ void __launch_bounds__(kScanBlock) doc_scan_kernel(const int32_t *__restrict__ pos, int64_t N,
+                                                             int32_t *__restrict__ doc_start,
+                                                             int32_t *__restrict__ block_agg,
+                                                             uint32_t *__restrict__ status)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;   // fresh status for this call
+    __shared__ int warp_max[kScanBlock / 32];
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
+    int v = (i < N && pos[i] == 0) ? static_cast<int>(i) : 0;
+    v = warp_incl_max(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 31) warp_max[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_max[lane];
+        w = warp_incl_max(w);
+        warp_max[lane] = w;
+    }
+    __syncthreads();
+    if (warp > 0) v = max(v, warp_max[warp - 1]);
+    if (i < N) doc_start[i] = v;
+    if (threadIdx.x == kScanBlock - 1) block_agg[blockIdx.x] = v;
+}
+
+// Adds the carry of all earlier blocks and records each query tile's first key.
+__global__ void __launch_bounds__(kScanBlock) doc_fixup_kernel(int64_t N, int32_t *__restrict__ doc_start,
+                                                              const int32_t *__restrict__ block_agg,
+                                                              int32_t *__restrict__ tile_lo)
+{
+    __shared__ int red[kScanBlock / 32];
+    int c = 0;
+    for (int b = threadIdx.x; b < static_cast<int>(blockIdx.x); b += kScanBlock) c = max(c, block_agg[b]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c = max(c, __shfl_xor_sync(0xffffffffu, c, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int w = red[threadIdx.x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
+        if (threadIdx.x == 0) red[0] = w;
+    }
+    __syncthreads();
+    const int carry = red[0];
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
+    if (i < N) {
+        const int v = max(doc_start[i], carry);
+        doc_start[i] = v;
+        if ((i % kTileM) == 0) tile_lo[i / kTileM] = v;
+    }
+}
+
+// For key tile t: one past the last query row whose document reaches a key of
+// the tile, i.e. the number of rows i with doc_start[i] <= min(t*128+127, N-1).
+__global__ void kv_qend_kernel(int64_t N, int T, const int32_t *__restrict__ doc_start, int32_t *__restrict__ kv_qend)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const int64_t last_key = min(static_cast<int64_t>(t) * kTileN + kTileN - 1, N - 1);
+    int64_t lo = last_key, hi = N;   // doc_start[last_key] <= last_key always holds
+    while (hi - lo > 1) {            // invariant: doc_start[lo] <= last_key, doc_start[hi] > last_key (or hi == N)
+        const int64_t mid = (lo + hi) >> 1;
+        if (doc_start[mid] <= last_key) lo = mid; else hi = mid;
+    }
+    kv_qend[t] = static_cast<int32_t>(hi);
+}
+
+// Counting sort of T tiles by work, heaviest first. Work of query tile t is
+// the number of key tiles it visits; work of key tile t is the number of query
+// tiles that visit it. One CTA; hist lives in global scratch [T + 1].
+template <bool kKeyTiles>
+__global__ void __launch_bounds__(1024) tile_order_kernel(int T, const int32_t *__restrict__ src,
+                                                         int32_t *__restrict__ hist, int32_t *__restrict__ order)
+{
+    __shared__ int part[1024];
+    const int tid = threadIdx.x;
+    for (int w = tid; w <= T; w += 1024) hist[w] = 0;
+    __syncthreads();
+    for (int t = tid; t < T; t += 1024) {
+        const int w = kKeyTiles ? (static_cast<int>((src[t] + kTileM - 1) / kTileM) - t)
+                                : (t - src[t] / kTileN + 1);
+        atomicAdd(&hist[w], 1);
+    }
+    __syncthreads();
+    // Exclusive prefix over work values in DESCENDING order:
+    // start[w] = number of tiles with work > w. Thread tid owns a contiguous
+    // segment of work values counted from the top.
+    const int per = (T + 1 + 1023) / 1024;
+    const int hi = T - tid * per;            // segment covers work values hi, hi-1, ..., hi-per+1
+    int sum = 0;
+    for (int k = 0; k < per; ++k) {
+        const int w = hi - k;
+        if (w >= 0) sum += hist[w];
+    }
+    part[tid] = sum;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        const int add = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += add;
+        __syncthreads();
+    }
+    int run = part[tid] - sum;   // tiles with work above this segment
+    for (int k = 0; k < per; ++k) {
+        const int w = hi - k;
+        if (w >= 0) {
+            const int c = hist[w];
+            hist[w] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    for (int t = tid; t < T; t += 1024) {
+        const int w = kKeyTiles ? (static_cast<int>((src[t] + kTileM - 1) / kTileM) - t)
+                                : (t - src[t] / kTileN + 1);
+        const int p = atomicAdd(&hist[w], 1);
+        order[p] = t;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
+                             cudaStream_t stream)
+{
+    const int64_t T = ceil_div(N, kTileM);
+    const int nb = static_cast<int>(ceil_div(N, kScanBlock));
+    int32_t *doc_start = reinterpret_cast<int32_t *>(ws + L.doc_start);
+    int32_t *tile_lo = reinterpret_cast<int32_t *>(ws + L.tile_lo);
+    int32_t *block_agg = reinterpret_cast<int32_t *>(ws + L.block_agg);
+    int32_t *scratch = reinterpret_cast<int32_t *>(ws + L.scratch);
+    doc_scan_kernel<<<nb, kScanBlock, 0, stream>>>(pos, N, doc_start, block_agg,
+                                                   reinterpret_cast<uint32_t *>(ws + L.status));
+    doc_fixup_kernel<<<nb, kScanBlock, 0, stream>>>(N, doc_start, block_agg, tile_lo);
+    tile_order_kernel<false><<<1, 1024, 0, stream>>>(static_cast<int>(T), tile_lo, scratch,
+                                                     reinterpret_cast<int32_t *>(ws + L.q_order));
+    if (backward) {
+        int32_t *kv_qend = reinterpret_cast<int32_t *>(ws + L.kv_qend);
+        kv_qend_kernel<<<static_cast<int>(ceil_div(T, 256)), 256, 0, stream>>>(N, static_cast<int>(T), doc_start,
+                                                                               kv_qend);
+        tile_order_kernel<true><<<1, 1024, 0, stream>>>(static_cast<int>(T), kv_qend, scratch,
+                                                        reinterpret_cast<int32_t *>(ws + L.kv_order));
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace uly

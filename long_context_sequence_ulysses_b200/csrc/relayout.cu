@@ -1,0 +1,141 @@
+// relayout.cu -- the two Ulysses all-to-all exchanges emulated on one GPU as
+// in-HBM permutations of 16-byte vectors.
+//
+// Sequence-to-head (page "Hugging Face并行加速：10倍提升超长序列训练效率", section
+// "Ulysses的工作原理", step 全体间通信): rank i's buffer [N/P][Hx][d] holds tokens
+// [i*N/P, (i+1)*N/P) for all heads; afterwards rank r holds [N][Hx/P][d], the
+// whole sequence for heads [r*Hx/P, (r+1)*Hx/P). Head-to-sequence (step
+// 全体间通信复原) is the inverse.
+//
+// For a fixed destination rank r and token n the data moved is one contiguous
+// chunk of C = Hx/P*d*2 bytes on both sides, so each CTA streams the chunks of
+// consecutive tokens: the chunk-side run is contiguous, the sequence-side
+// rows are strided by Hx*d*2 bytes. Threads are mapped once to (token offset,
+// vector within chunk), so the inner loop has no integer division.
+#include "ulysses_internal.cuh"
+
+namespace uly {
+
+namespace {
+
+constexpr int kRelayoutThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v)
+{
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// One kernel for both directions.
+//   seq side  : row n of the sequence layout, vector (r*C + e) of its Hx*d/8 vectors
+//   head side : row n of rank r's slice, vector e of its C vectors
+// to_head = true copies seq -> head, false copies head -> seq.
+// ranks: gridDim.y ranks starting at rank0; head_rank_stride is the distance
+// (in vectors) between consecutive ranks' slices on the head side (N*C for
+// the all-ranks layout, 0 when a single rank's slice is given).
+struct RelayoutArgs {
+    const uint4 *src;
+    uint4 *dst;
+    int64_t N;          // tokens
+    int64_t row_vecs;   // Hx*d/8: vectors per token row on the sequence side
+    int C;              // Hx/P*d/8: vectors per chunk
+    int rank0;
+    int64_t head_rank_stride;
+    int tokens_per_iter;  // tokens covered by one CTA pass (kRelayoutThreads / C, >= 1)
+    int e_iters;          // chunks wider than the CTA: ceil(C / kRelayoutThreads)
+};
+
+template <bool kToHead>
+__global__ void __launch_bounds__(kRelayoutThreads) relayout_kernel(RelayoutArgs a)
+{
+    const int r = a.rank0 + blockIdx.y;
+    const int t = threadIdx.x;
+    int tok_off, e0;
+    if (a.e_iters == 1) {
+        tok_off = t / a.C;
+        e0 = t - tok_off * a.C;
+        if (tok_off >= a.tokens_per_iter) return;
+    } else {
+        tok_off = 0;
+        e0 = t;
+    }
+    const int64_t head_base = (blockIdx.y) * a.head_rank_stride;
+    const int64_t seq_col = static_cast<int64_t>(r) * a.C;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * a.tokens_per_iter;
+
+    for (int ei = 0; ei < a.e_iters; ++ei) {
+        const int e = e0 + ei * kRelayoutThreads;
+        if (e >= a.C) break;
+        int64_t n = static_cast<int64_t>(blockIdx.x) * a.tokens_per_iter + tok_off;
+        for (; n < a.N; n += kUnroll * step) {
+            uint4 v[kUnroll];
+            int64_t nn[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                nn[u] = n + u * step;
+                if (nn[u] < a.N) {
+                    const int64_t s_off = kToHead ? nn[u] * a.row_vecs + seq_col + e
+                                                  : head_base + nn[u] * a.C + e;
+                    v[u] = ld_stream(a.src + s_off);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (nn[u] < a.N) {
+                    const int64_t d_off = kToHead ? head_base + nn[u] * a.C + e
+                                                  : nn[u] * a.row_vecs + seq_col + e;
+                    st_stream(a.dst + d_off, v[u]);
+                }
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_relayout(bool to_head, const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
+                            cudaStream_t stream, int num_sms)
+{
+    RelayoutArgs a;
+    a.src = static_cast<const uint4 *>(src);
+    a.dst = static_cast<uint4 *>(dst);
+    a.N = N;
+    a.row_vecs = static_cast<int64_t>(Hx) * d / 8;
+    a.C = (Hx / P) * d / 8;
+    const int nranks = rank < 0 ? P : 1;
+    a.rank0 = rank < 0 ? 0 : rank;
+    a.head_rank_stride = rank < 0 ? N * a.C : 0;
+    if (a.C <= kRelayoutThreads) {
+        a.tokens_per_iter = kRelayoutThreads / a.C;
+        a.e_iters = 1;
+    } else {
+        a.tokens_per_iter = 1;
+        a.e_iters = (a.C + kRelayoutThreads - 1) / kRelayoutThreads;
+    }
+    const int64_t groups = (N + a.tokens_per_iter - 1) / a.tokens_per_iter;
+    // Enough CTAs to fill every SM several times over, each streaming kUnroll
+    // independent vectors per thread per pass.
+    const int64_t want = (groups + kUnroll - 1) / kUnroll;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    const int64_t per_rank_cap = (cap + nranks - 1) / nranks;
+    int gx = static_cast<int>(want < per_rank_cap ? want : per_rank_cap);
+    if (gx < 1) gx = 1;
+    dim3 grid(gx, nranks);
+    if (to_head)
+        relayout_kernel<true><<<grid, kRelayoutThreads, 0, stream>>>(a);
+    else
+        relayout_kernel<false><<<grid, kRelayoutThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace uly

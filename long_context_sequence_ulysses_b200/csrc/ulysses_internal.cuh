@@ -1,0 +1,105 @@
+// ulysses_internal.cuh -- declarations shared by the library's .cu files:
+// workspace layout and kernel launchers. Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace uly {
+
+constexpr int kTileM = 128;   // query rows per tile
+constexpr int kTileN = 128;   // keys per tile
+constexpr int kScanBlock = 1024;
+constexpr uint32_t kStatusTimeoutHost = 1u;   // same bit as the device-side timeout flag
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace layout (every section 256-byte aligned):
+//   status     uint32 [64]        status word (bit 0: a bounded wait ran out)
+//   doc_start  int32  [N]         first token of the row's document
+//   tile_lo    int32  [T]         doc_start of the first row of each 128-row tile
+//   q_order    int32  [T]         query tiles, heaviest first
+//   block_agg  int32  [ceil(N/1024)]  per-block maxima of the doc-start scan
+//   scratch    int32  [T + 1]     histogram for the tile sort
+// backward only:
+//   kv_qend    int32  [T]         one past the last row that attends to key tile t
+//   kv_order   int32  [T]         key tiles, heaviest first
+//   delta      fp32   [Hl][N]     D_i = sum_c dO_ic O_ic
+struct WsLayout {
+    size_t status, doc_start, tile_lo, q_order, block_agg, scratch;
+    size_t kv_qend, kv_order, delta;
+    size_t total;
+};
+
+inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
+{
+    WsLayout L{};
+    const int64_t T = ceil_div(N, kTileM);
+    const int64_t nb = ceil_div(N, kScanBlock);
+    size_t off = 0;
+    L.status = off;    off += align256(64 * 4);
+    L.doc_start = off; off += align256(static_cast<size_t>(N) * 4);
+    L.tile_lo = off;   off += align256(static_cast<size_t>(T) * 4);
+    L.q_order = off;   off += align256(static_cast<size_t>(T) * 4);
+    L.block_agg = off; off += align256(static_cast<size_t>(nb) * 4);
+    L.scratch = off;   off += align256(static_cast<size_t>(T + 1) * 4);
+    if (backward) {
+        L.kv_qend = off;  off += align256(static_cast<size_t>(T) * 4);
+        L.kv_order = off; off += align256(static_cast<size_t>(T) * 4);
+        L.delta = off;    off += align256(static_cast<size_t>(N) * Hl * 4);
+    } else {
+        L.kv_qend = L.kv_order = L.delta = 0;
+    }
+    L.total = off;
+    return L;
+}
+
+// relayout.cu
+cudaError_t launch_relayout(bool to_head, const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
+                            cudaStream_t stream, int num_sms);
+
+// docbounds.cu: doc_start, tile_lo and the query-tile order (and, when
+// backward, kv_qend and the key-tile order).
+cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
+                             cudaStream_t stream);   // also clears the status word
+
+// Forward attention launch description.
+struct FwdLaunch {
+    const void *q, *k, *v;       // base pointers of [N][Hq_total][d] / [N][Hkv_total][d]
+    int Hq_total, Hkv_total;     // heads per token row in the q / kv buffers
+    int q_head0, kv_head0;       // first head of this rank's slice in those rows
+    void *o;                     // base of [N][Ho_total][d]
+    int Ho_total, o_head0;
+    float *lse;                  // [Hl][N]
+    int64_t N;
+    int Hl, Hkvl, d;
+    float scale;
+    const char *ws;
+    WsLayout L;
+    uint64_t wait_limit_ns;
+};
+cudaError_t launch_attn_fwd(const FwdLaunch &a, cudaStream_t stream);
+
+// Backward attention launch description (no fused layout: slice buffers).
+struct BwdLaunch {
+    const void *q, *k, *v, *o, *dout;
+    const float *lse;
+    void *dq, *dk, *dv;
+    int64_t N;
+    int Hl, Hkvl, d;
+    float scale;
+    char *ws;
+    WsLayout L;
+    uint64_t wait_limit_ns;
+};
+cudaError_t launch_attn_bwd(const BwdLaunch &a, cudaStream_t stream);
+
+// api.cu
+int num_sms_current_device();
+bool encode_tmap_3d(void *tmap /*CUtensorMap*/, const void *base, int64_t inner, int64_t mid, int64_t outer,
+                    int64_t mid_stride_bytes, int64_t outer_stride_bytes, int box_inner, int box_outer,
+                    int swizzle_bytes);
+
+}  // namespace uly

@@ -1,0 +1,45 @@
+"""Shared helpers for the parity tests (sampling rows, error metrics)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+# Acceptance thresholds for floating-point results against the fp64 oracle:
+# max-abs 2e-2 and mean-abs 2e-3 (bf16 inputs, fp32 accumulation, bf16 O).
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+
+
+def sample_rows(lengths, N: int, n_random: int, seed: int, cap_doc_edges: int = 64) -> np.ndarray:
+    """Stratified query rows: first/last row of documents (up to a cap), the
+    first/last row of 128-row tiles near them, the last row, plus uniform
+    random rows."""
+    rng = np.random.default_rng(seed)
+    rows = {0, N - 1}
+    starts = np.cumsum([0] + list(lengths))[:-1]
+    ends = starts + np.asarray(lengths) - 1
+    idx = np.arange(len(lengths))
+    if len(idx) > cap_doc_edges:
+        idx = np.sort(rng.choice(idx, cap_doc_edges, replace=False))
+    for t in idx:
+        rows.update([int(starts[t]), int(ends[t])])
+        rows.update([int(min(N - 1, (starts[t] // 128) * 128 + 127)), int(min(N - 1, starts[t] + 1))])
+    rows.update(rng.integers(0, N, size=n_random).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int64)
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def err_stats(got: np.ndarray, ref: np.ndarray):
+    d = np.abs(got.astype(np.float64) - ref)
+    return float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0
+
+
+def assert_close(name: str, got: np.ndarray, ref: np.ndarray, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    mx, mn = err_stats(got, ref)
+    assert mx <= max_abs and mn <= mean_abs, f"{name}: max-abs {mx:.3e} (<= {max_abs}), mean-abs {mn:.3e} (<= {mean_abs})"
+    return mx, mn

@@ -1,0 +1,138 @@
+"""Parity of the tensor-core attention forward with the fp64 oracle.
+
+Small cases are compared on every row (several 128-row tiles, ragged tails,
+packed documents, GQA, every supported head dimension); the five workloads
+are compared on stratified samples of rows (each sampled row exact over all
+its keys), through the same launch the benchmark times."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_close, bf16_to_f64, sample_rows
+from workloads import WORKLOADS, make_inputs, random_case
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(c, scale=None):
+    import long_context_sequence_ulysses_b200 as U
+    o, lse = U.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"], scale=scale)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+CASES = [
+    # (lengths, Hl, Hkvl, d)
+    ([256], 2, 2, 32),
+    ([128], 1, 1, 128),
+    ([1], 1, 1, 128),
+    ([300], 2, 1, 128),               # ragged tail
+    ([1000], 4, 1, 128),
+    ([700, 1, 300, 23, 200], 4, 2, 128),
+    ([5] * 60, 2, 2, 64),             # many short documents inside one tile
+    ([129, 127, 384, 2], 8, 2, 64),
+    ([513, 511], 4, 4, 32),
+    ([2048], 1, 1, 64),
+    ([3000, 1500, 2], 2, 1, 128),
+]
+
+
+@pytest.mark.parametrize("lengths,Hl,Hkvl,d", CASES)
+def test_fwd_matches_oracle_all_rows(lengths, Hl, Hkvl, d):
+    N = sum(lengths)
+    c = random_case(N, Hl, Hkvl, d, lengths, seed=N + 7 * Hl + d, device="cuda")
+    o, lse = _run(c)
+    ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    assert_close("O", bf16_to_f64(o), ro)
+    assert_close("LSE", lse.double().cpu().numpy(), rl)
+
+
+def test_fwd_scale_argument():
+    lengths = [400, 100]
+    c = random_case(500, 2, 1, 128, lengths, seed=3, device="cuda")
+    o, lse = _run(c, scale=0.05)
+    ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"], scale=0.05)
+    assert_close("O", bf16_to_f64(o), ro)
+    assert_close("LSE", lse.double().cpu().numpy(), rl)
+
+
+def test_fwd_one_token_documents_return_v():
+    N, Hl, Hkvl, d = 384, 4, 2, 128
+    c = random_case(N, Hl, Hkvl, d, [1] * N, seed=1, device="cuda")
+    o, lse = _run(c)
+    v = c["v"].repeat_interleave(Hl // Hkvl, dim=1)
+    assert torch.equal(o, v)          # one key: weight exactly 1, O is V rounded back to bf16
+
+
+def test_fwd_uniform_v():
+    lengths = [200, 50, 262]
+    N = sum(lengths)
+    c = random_case(N, 2, 1, 64, lengths, seed=2, device="cuda")
+    c["v"][:] = torch.linspace(-2, 2, 64, device="cuda").to(torch.bfloat16)
+    o, _ = _run(c)
+    ref = c["v"][0, 0].float().expand(N, 2, 64)
+    assert (o.float() - ref).abs().max().item() <= 2e-2
+
+
+def test_fwd_deterministic_and_fused_equals_unfused():
+    import long_context_sequence_ulysses_b200 as U
+    lengths = [600, 424]
+    N, P, H, Hkv, d = 1024, 4, 8, 4, 128
+    c = random_case(N, H, Hkv, d, lengths, seed=5, device="cuda")
+    o_seq = torch.zeros_like(c["q"])
+    for r in range(P):
+        qs = U.seq_to_head(c["q"], P, rank=r)
+        ks = U.seq_to_head(c["k"], P, rank=r)
+        vs = U.seq_to_head(c["v"], P, rank=r)
+        o1, l1 = U.attn_fwd(qs, ks, vs, c["position_ids"])
+        o2, l2 = U.attn_fwd(qs, ks, vs, c["position_ids"])
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        o3 = torch.zeros_like(c["q"])
+        _, l3 = U.attn_fwd_fused(c["q"], c["k"], c["v"], c["position_ids"], P, r, out=o3)
+        assert torch.equal(o3[:, r * H // P:(r + 1) * H // P], o1) and torch.equal(l3, l1)
+        U.attn_fwd_fused(c["q"], c["k"], c["v"], c["position_ids"], P, r, out=o_seq)
+    # sharded (all ranks, fused) equals unsharded attention on all heads at once
+    o_all, _ = U.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    assert torch.equal(o_seq, o_all)
+
+
+def test_fwd_empty():
+    import long_context_sequence_ulysses_b200 as U
+    z = torch.empty((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    o, lse = U.attn_fwd(z, z[:, :1], z[:, :1], torch.empty(0, dtype=torch.int32, device="cuda"))
+    assert o.shape == (0, 2, 128) and lse.shape == (2, 0)
+
+
+WORKLOAD_SAMPLES = {"tiny": None, "llama8b": 160, "long131k": 24, "million": 6, "train": 160}
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama8b", "long131k", "million", "train"])
+def test_workload_forward(name):
+    """Rank 0's head slice of each workload, produced by the seq->head exchange
+    and run through the same forward launch the benchmark times."""
+    import long_context_sequence_ulysses_b200 as U
+    w = WORKLOADS[name]
+    inp = make_inputs(w, device="cuda", with_grad_out=False)
+    rank = 0
+    q = U.seq_to_head(inp["q"], w.P, rank=rank)
+    k = U.seq_to_head(inp["k"], w.P, rank=rank)
+    v = U.seq_to_head(inp["v"], w.P, rank=rank)
+    del inp["q"], inp["k"], inp["v"]
+    o, lse = U.attn_fwd(q, k, v, inp["position_ids"])
+    torch.cuda.synchronize()
+    n_rand = WORKLOAD_SAMPLES[name]
+    if n_rand is None:
+        rows = np.arange(w.N)
+    else:
+        rows = sample_rows(inp["lengths"], w.N, n_rand, seed=w.seed)
+        if name in ("long131k", "million"):
+            # single long document: keep the sample affordable but include the far end
+            rng = np.random.default_rng(w.seed)
+            rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1], rng.integers(0, w.N, n_rand)]))
+    rt = torch.from_numpy(rows).cuda()
+    ro, rl = oracle.attn_fwd(q.cpu(), k.cpu(), v.cpu(), inp["position_ids"].cpu(), rows=rows)
+    assert_close("O", bf16_to_f64(o[rt]), ro)
+    assert_close("LSE", lse[:, rt].double().cpu().numpy(), rl)
