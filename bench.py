@@ -39,6 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+BWD_LAUNCHES = 8   # doc-bounds (5) + delta, dK/dV and dQ kernels
 
 
 def load_peaks():
@@ -170,17 +171,17 @@ def run_gpu(args):
     Hl, Hkvl, d, N = w.Hl, w.Hkvl, w.d, w.N
     pairs, fwd_flop, bwd_flop, relayout_bytes = workload_work(w, lengths)
 
-    # rank-slice buffers, reused by every emulated rank
-    qs = torch.empty((N, Hl, d), dtype=torch.bfloat16, device=dev)
-    ks = torch.empty((N, Hkvl, d), dtype=torch.bfloat16, device=dev)
-    vs = torch.empty((N, Hkvl, d), dtype=torch.bfloat16, device=dev)
-    os_ = torch.empty((N, Hl, d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((Hl, N), dtype=torch.float32, device=dev)
+    # head-slice buffers of all emulated ranks: [P][N][H/P][d]
+    q_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
+    k_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    o_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
+    lse_all = torch.empty((P * Hl, N), dtype=torch.float32, device=dev)
     o_seq = torch.empty_like(q_seq)
     ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
     if w.backward:
-        dos = torch.empty_like(qs)
-        dqs, dks, dvs = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
+        do_all = torch.empty_like(q_all)
+        dq_all, dk_all, dv_all = torch.empty_like(q_all), torch.empty_like(k_all), torch.empty_like(v_all)
         dq_seq, dk_seq, dv_seq = torch.empty_like(q_seq), torch.empty_like(k_seq), torch.empty_like(v_seq)
 
     stream = torch.cuda.current_stream(dev)
@@ -199,23 +200,32 @@ def run_gpu(args):
             fn()
 
     def step(record: bool):
+        # first all-to-all: every rank's head slice of Q, K, V
+        timed("relayout", lambda: U.seq_to_head(q_seq, P, out=q_all))
+        timed("relayout", lambda: U.seq_to_head(k_seq, P, out=k_all))
+        timed("relayout", lambda: U.seq_to_head(v_seq, P, out=v_all))
+        n = 3
         for r in range(P):
-            timed("relayout", lambda: U.seq_to_head(q_seq, P, rank=r, out=qs))
-            timed("relayout", lambda: U.seq_to_head(k_seq, P, rank=r, out=ks))
-            timed("relayout", lambda: U.seq_to_head(v_seq, P, rank=r, out=vs))
-            timed("attn_fwd", lambda: U.attn_fwd(qs, ks, vs, pos, out=os_, lse=lse, ws=ws))
-            n = 3 + 4
-            if w.backward:
-                timed("relayout", lambda: U.seq_to_head(do_seq, P, rank=r, out=dos))
-                timed("attn_bwd", lambda: U.attn_bwd(qs, ks, vs, os_, dos, lse, pos, ws=ws, dq=dqs, dk=dks, dv=dvs))
-                timed("relayout", lambda: U.head_to_seq(dqs, P, rank=r, out=dq_seq))
-                timed("relayout", lambda: U.head_to_seq(dks, P, rank=r, out=dk_seq))
-                timed("relayout", lambda: U.head_to_seq(dvs, P, rank=r, out=dv_seq))
-                n += 1 + 8 + 3
-            timed("relayout", lambda: U.head_to_seq(os_, P, rank=r, out=o_seq))
+            timed("attn_fwd", lambda: U.attn_fwd(q_all[r], k_all[r], v_all[r], pos, out=o_all[r],
+                                                 lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws))
+            n += 4
+        if w.backward:
+            timed("relayout", lambda: U.seq_to_head(do_seq, P, out=do_all))
             n += 1
-            if record:
-                launches["n"] += n
+            for r in range(P):
+                timed("attn_bwd", lambda: U.attn_bwd(q_all[r], k_all[r], v_all[r], o_all[r], do_all[r],
+                                                     lse_all[r * Hl:(r + 1) * Hl], pos, ws=ws, dq=dq_all[r],
+                                                     dk=dk_all[r], dv=dv_all[r]))
+                n += BWD_LAUNCHES
+            timed("relayout", lambda: U.head_to_seq(dq_all, P, out=dq_seq))
+            timed("relayout", lambda: U.head_to_seq(dk_all, P, out=dk_seq))
+            timed("relayout", lambda: U.head_to_seq(dv_all, P, out=dv_seq))
+            n += 3
+        # second all-to-all: O back to sequence shards
+        timed("relayout", lambda: U.head_to_seq(o_all, P, out=o_seq))
+        n += 1
+        if record:
+            launches["n"] += n
 
     # warm-up
     saved = args.kernel_events
@@ -287,8 +297,9 @@ def run_gpu(args):
         "config": {
             "workload": w.name, "N": N, "P": P, "H": w.H, "Hkv": w.Hkv, "d": d, "docs": w.docs,
             "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
-            "step": "for each of P emulated ranks: seq_to_head(Q,K,V) + attn_fwd" + (" + attn_bwd" if w.backward else "")
-                    + " + head_to_seq(O)",
+            "step": "seq_to_head(Q,K,V) for all P ranks; attn_fwd for each rank's head slice"
+                    + ("; seq_to_head(dO), attn_bwd per rank, head_to_seq(dQ,dK,dV)" if w.backward else "")
+                    + "; head_to_seq(O) for all ranks",
             "l2": "inputs larger than L2 (126 MB): Q alone is %d MiB" % (N * w.H * d * 2 >> 20),
         },
         "roofline": {
@@ -328,60 +339,59 @@ def run_gpu(args):
 
 def run_e2e(U, w, inp, args, dev):
     """Same step through the public API from pinned HOST buffers: each step
-    copies Q, K, V and position ids host->device and reads O and LSE back."""
-    P, N, d = w.P, w.N, w.d
-    hq = inp["q"].cpu().pin_memory()
-    hk = inp["k"].cpu().pin_memory()
-    hv = inp["v"].cpu().pin_memory()
-    hpos = inp["position_ids"].cpu().pin_memory()
-    hdo = inp["do"].cpu().pin_memory() if w.backward else None
+    copies Q, K, V (and dO) and the position ids host->device, runs the path,
+    and reads O and LSE (and dQ, dK, dV) back to the host."""
+    P, N, d, Hl, Hkvl = w.P, w.N, w.d, w.Hl, w.Hkvl
+    pin = lambda t: t.cpu().pin_memory()
+    hq, hk, hv, hpos = pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), pin(inp["position_ids"])
+    hdo = pin(inp["do"]) if w.backward else None
     ho = torch.empty_like(hq).pin_memory()
     hlse = torch.empty((w.H, N), dtype=torch.float32).pin_memory()
-    dq_, dk_, dv_ = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
-    o_seq = torch.empty_like(inp["q"])
-    lse_all = torch.empty((w.H, N), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    ws = torch.empty(U.workspace_bytes(N, w.Hl, w.Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
-    qs = torch.empty((N, w.Hl, d), dtype=torch.bfloat16, device=dev)
-    ks = torch.empty((N, w.Hkvl, d), dtype=torch.bfloat16, device=dev)
-    vs = torch.empty_like(ks)
-    os_ = torch.empty_like(qs)
-    dq_s, dk_s, dv_s, do_s = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(ks), torch.empty_like(qs)
     gq, gk, gv = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
     gpos = torch.empty_like(inp["position_ids"])
-    gdo = torch.empty_like(inp["q"]) if w.backward else None
-    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hpos.numel() * 4 + (hdo.numel() * 2 if w.backward else 0)
-    d2h = ho.numel() * 2 + hlse.numel() * 4 + ((hq.numel() + 2 * hk.numel()) * 2 if w.backward else 0)
-    hdq = torch.empty_like(hq).pin_memory() if w.backward else None
-    hdk = torch.empty_like(hk).pin_memory() if w.backward else None
-    hdv = torch.empty_like(hv).pin_memory() if w.backward else None
+    q_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
+    k_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty_like(k_all)
+    o_all = torch.empty_like(q_all)
+    lse_all = torch.empty((w.H, N), dtype=torch.float32, device=dev)
+    o_seq = torch.empty_like(gq)
+    ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
+    if w.backward:
+        gdo = torch.empty_like(gq)
+        do_all, dq_all = torch.empty_like(q_all), torch.empty_like(q_all)
+        dk_all, dv_all = torch.empty_like(k_all), torch.empty_like(k_all)
+        dq_seq, dk_seq, dv_seq = torch.empty_like(gq), torch.empty_like(gk), torch.empty_like(gv)
+        hdq, hdk, hdv = (torch.empty_like(hq).pin_memory(), torch.empty_like(hk).pin_memory(),
+                         torch.empty_like(hv).pin_memory())
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2 + hpos.numel() * 4 + (hdo.numel() * 2 if w.backward else 0)
+    d2h = ho.numel() * 2 + hlse.numel() * 4 + ((hq.numel() + hk.numel() + hv.numel()) * 2 if w.backward else 0)
+    stream = torch.cuda.current_stream(dev)
 
     def step():
         gq.copy_(hq, non_blocking=True)
         gk.copy_(hk, non_blocking=True)
         gv.copy_(hv, non_blocking=True)
         gpos.copy_(hpos, non_blocking=True)
+        U.seq_to_head(gq, P, out=q_all)
+        U.seq_to_head(gk, P, out=k_all)
+        U.seq_to_head(gv, P, out=v_all)
+        for r in range(P):
+            U.attn_fwd(q_all[r], k_all[r], v_all[r], gpos, out=o_all[r], lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws)
         if w.backward:
             gdo.copy_(hdo, non_blocking=True)
-        for r in range(P):
-            U.seq_to_head(gq, P, rank=r, out=qs)
-            U.seq_to_head(gk, P, rank=r, out=ks)
-            U.seq_to_head(gv, P, rank=r, out=vs)
-            U.attn_fwd(qs, ks, vs, gpos, out=os_, lse=lse_all[r * w.Hl:(r + 1) * w.Hl], ws=ws)
-            if w.backward:
-                U.seq_to_head(gdo, P, rank=r, out=do_s)
-                U.attn_bwd(qs, ks, vs, os_, do_s, lse_all[r * w.Hl:(r + 1) * w.Hl], gpos, ws=ws, dq=dq_s, dk=dk_s,
-                           dv=dv_s)
-                U.head_to_seq(dq_s, P, rank=r, out=dq_)
-                U.head_to_seq(dk_s, P, rank=r, out=dk_)
-                U.head_to_seq(dv_s, P, rank=r, out=dv_)
-            U.head_to_seq(os_, P, rank=r, out=o_seq)
+            U.seq_to_head(gdo, P, out=do_all)
+            for r in range(P):
+                U.attn_bwd(q_all[r], k_all[r], v_all[r], o_all[r], do_all[r], lse_all[r * Hl:(r + 1) * Hl], gpos,
+                           ws=ws, dq=dq_all[r], dk=dk_all[r], dv=dv_all[r])
+            U.head_to_seq(dq_all, P, out=dq_seq)
+            U.head_to_seq(dk_all, P, out=dk_seq)
+            U.head_to_seq(dv_all, P, out=dv_seq)
+            hdq.copy_(dq_seq, non_blocking=True)
+            hdk.copy_(dk_seq, non_blocking=True)
+            hdv.copy_(dv_seq, non_blocking=True)
+        U.head_to_seq(o_all, P, out=o_seq)
         ho.copy_(o_seq, non_blocking=True)
         hlse.copy_(lse_all, non_blocking=True)
-        if w.backward:
-            hdq.copy_(dq_, non_blocking=True)
-            hdk.copy_(dk_, non_blocking=True)
-            hdv.copy_(dv_, non_blocking=True)
 
     for _ in range(2):
         step()
