@@ -139,6 +139,26 @@ int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o,
                      void *dq, void *dk, void *dv, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * No counterpart in the pages: ulysses_attn_fwd for callers that cannot
+ * allocate device memory, such as a plugin inside a host framework that owns
+ * all device memory through its own pool and hands over only input and output
+ * buffers, or a latency-critical path that must not call cudaMalloc (which can
+ * synchronise the device). Same arguments and results as ulysses_attn_fwd
+ * without the workspace: the scratch lives in a static device array inside the
+ * library (544 KiB, held by every GPU that loads the library until exit).
+ *  - N > 131072 returns ULYSSES_ERR_UNSUPPORTED.
+ *  - Nothing is allocated. The first call on each device looks up the array's
+ *    address (cudaGetSymbolAddress) with that device current; make that first
+ *    call before any stream capture.
+ *  - All calls on a device share the array; calls that overlap on the GPU
+ *    (different streams, unordered threads) race and give wrong results.
+ *  - A bounded device wait that runs out is not reported by this entry point.
+ */
+int ulysses_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                             const int32_t *position_ids, int64_t N, int Hl, int Hkvl, int d,
+                             float scale, void *o, float *lse, void *stream);
+
+/*
  * Synchronise `stream` and report the status the latest attention call left
  * in `ws`: ULYSSES_ERR_TIMEOUT if a bounded device wait ran out, else
  * ULYSSES_OK (or ULYSSES_ERR_CUDA if synchronisation failed). Clears the flag.

@@ -58,6 +58,8 @@ EncodeTiledFn encode_fn()
 
 }  // namespace
 
+int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 int num_sms_current_device()
 {
     static int cache[64] = {};
