@@ -1,9 +1,625 @@
-// attn_bwd.cu -- attention backward for one rank's head slice (placeholder
-// until the tensor-core kernels land).
+// attn_bwd.cu -- attention backward for one rank's head slice on the sm_100a
+// tensor cores: the gradients of sum(dO * O) with respect to Q, K and V.
+//
+// With s_ij = scale q_i.k_j, P_ij = exp(s_ij - LSE_i) (recomputed from the
+// forward's logsumexp), D_i = sum_c dO_ic O_ic:
+//   dV_j = sum_{h in group} sum_i P_ij dO_i          dP_ij = dO_i . v_j
+//   dS_ij = P_ij (dP_ij - D_i)
+//   dK_j = scale sum_{h in group} sum_i dS_ij q_i     dQ_i = scale sum_j dS_ij k_j
+// over the unmasked pairs (doc_start(i) <= j <= i). Training through the
+// attention step of Ulysses needs these (every page speaks of training; the
+// attention itself is the "本地注意力计算" step of the page "Hugging Face并行加速：
+// 10倍提升超长序列训练效率", section "Ulysses的工作原理").
+//
+// Three kernels, all deterministic (no atomics):
+//  1. prep: D_i and LSE_i*log2(e) per (head, row) into a 128-padded layout.
+//  2. dK/dV: one CTA per (key tile, KV head) loops over the query heads of the
+//     GQA group and the query tiles that see the key tile:
+//       S^T = K Q^T, dP^T = V dO^T       (SS MMA, M = keys, N = queries)
+//       P^T, dS^T -> bf16 into the first 64 columns of S^T / dP^T in TMEM
+//       dV += P^T dO, dK += dS^T Q      (TS MMA, dO / Q read MN-major)
+//     so the group reduction happens in the accumulator.
+//  3. dQ: one CTA per (query tile, head) loops over its key tiles:
+//       S = Q K^T, dP = dO V^T -> dS (bf16, into S's columns) -> dQ += dS K.
+#include "ptx.cuh"
 #include "ulysses_internal.cuh"
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
 
 namespace uly {
 
-cudaError_t launch_attn_bwd(const BwdLaunch &, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kBwdThreads = 256;
+constexpr int kComputeWarp0 = 4;   // warps 4..7: the compute warpgroup (TMEM lanes 0..127)
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+    const int32_t *doc_start;
+    const int32_t *tile_lo;
+    const int32_t *q_order;
+    const int32_t *kv_qend;
+    const int32_t *kv_order;
+    const float *delta;   // [Hl][Npad]
+    const float *lse2;    // [Hl][Npad]
+    __nv_bfloat16 *dq, *dk, *dv;
+    int N, Npad, T, Hl, Hkvl;
+    float scale_log2, scale;
+    uint32_t *status;
+    uint64_t wait_limit_ns;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int SW = (D * 2 >= 128) ? 128 : D * 2;
+    static constexpr int AW = SW / 2;
+    static constexpr int NA = D / AW;
+    static constexpr int ATOM_BYTES = kTileM * SW;
+    static constexpr int TILE_BYTES = kTileM * D * 2;
+    static constexpr int NST = 2;
+    static constexpr uint32_t SWZ = (SW == 128) ? kSwizzle128 : kSwizzle64;
+    static constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false, false);
+    static constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, false, true);
+    static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
+    // dK/dV kernel shared memory: K, V, then NST stages of {Q, dO}, then
+    // NST stages of {lse2 row, delta row} (512 bytes each), then barriers.
+    static constexpr int KV_OFF_K = 0;
+    static constexpr int KV_OFF_V = TILE_BYTES;
+    static constexpr int KV_OFF_Q = 2 * TILE_BYTES;
+    static constexpr int KV_OFF_DO = KV_OFF_Q + NST * TILE_BYTES;
+    static constexpr int KV_OFF_ROW = KV_OFF_DO + NST * TILE_BYTES;
+    static constexpr int KV_OFF_BAR = KV_OFF_ROW + NST * 2 * 512;
+    static constexpr int KV_SMEM = KV_OFF_BAR + 16 * 8 + 16 + 1024;
+    // dQ kernel shared memory: Q, dO, then NST stages of {K, V}, then barriers.
+    static constexpr int Q_OFF_Q = 0;
+    static constexpr int Q_OFF_DO = TILE_BYTES;
+    static constexpr int Q_OFF_K = 2 * TILE_BYTES;
+    static constexpr int Q_OFF_V = Q_OFF_K + NST * TILE_BYTES;
+    static constexpr int Q_OFF_BAR = Q_OFF_V + NST * TILE_BYTES;
+    static constexpr int Q_SMEM = Q_OFF_BAR + 16 * 8 + 16 + 1024;
+};
+
+__device__ __forceinline__ float dot8_bf16(const uint4 &a, const uint4 &b)
+{
+    const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
+    const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 fx = __bfloat1622float2(x[k]);
+        const float2 fy = __bfloat1622float2(y[k]);
+        acc = fmaf(fx.x, fy.x, acc);
+        acc = fmaf(fx.y, fy.y, acc);
+    }
+    return acc;
+}
+
+// D_i = sum_c dO_ic O_ic and LSE_i * log2(e), one warp per (head, padded row).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                      const __nv_bfloat16 *__restrict__ dout,
+                                                      const float *__restrict__ lse, float *__restrict__ delta,
+                                                      float *__restrict__ lse2, int N, int Npad, int Hl)
+{
+    const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= static_cast<int64_t>(Hl) * Npad) return;
+    const int h = static_cast<int>(w / Npad);
+    const int i = static_cast<int>(w % Npad);
+    float acc = 0.f;
+    if (i < N) {
+        const uint4 *po = reinterpret_cast<const uint4 *>(o + (static_cast<int64_t>(i) * Hl + h) * D);
+        const uint4 *pd = reinterpret_cast<const uint4 *>(dout + (static_cast<int64_t>(i) * Hl + h) * D);
+        for (int v = lane; v < D / 8; v += 32) acc += dot8_bf16(po[v], pd[v]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        delta[w] = i < N ? acc : 0.f;
+        lse2[w] = i < N ? lse[static_cast<int64_t>(h) * N + i] * kLog2e : CUDART_INF_F;
+    }
+}
+
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// K-major SS descriptors for a 16-element K step kk of a 128-row tile.
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int kk)
+{
+    using C = BwdCfg<D>;
+    constexpr int steps = C::SW / 32;
+    const uint32_t koff = (kk / steps) * C::ATOM_BYTES + (kk % steps) * 32;
+    return smem_desc(tile_addr + koff, 16, 8 * C::SW, C::SWZ);
+}
+
+// MN-major descriptor of a [rows][d] tile used as B with N = d, K = rows:
+// 16 rows per K step.
+template <int D>
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk)
+{
+    using C = BwdCfg<D>;
+    return smem_desc(tile_addr + kk * 16 * C::SW, C::ATOM_BYTES, 8 * C::SW, C::SWZ);
+}
+
+template <int D>
+__device__ __forceinline__ void tma_tile(const CUtensorMap *m, uint8_t *dst, uint64_t *bar, int head, int row0)
+{
+    using C = BwdCfg<D>;
+#pragma unroll
+    for (int a = 0; a < C::NA; ++a) tma_load_3d(dst + a * C::ATOM_BYTES, m, bar, a * C::AW, head, row0);
+}
+
+// ============================================================== dK / dV
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                         const BwdParams p)
+{
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sK = smem + C::KV_OFF_K;
+    uint8_t *sV = smem + C::KV_OFF_V;
+    uint8_t *sQ = smem + C::KV_OFF_Q;
+    uint8_t *sDO = smem + C::KV_OFF_DO;
+    float *sRow = reinterpret_cast<float *>(smem + C::KV_OFF_ROW);   // [NST][2][128]: lse2, delta
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::KV_OFF_BAR);
+    uint64_t *kv_full = bars;
+    uint64_t *qdo_full = bars + 1;            // [NST]
+    uint64_t *qdo_empty = qdo_full + C::NST;  // [NST]
+    uint64_t *s_full = qdo_empty + C::NST;
+    uint64_t *ds_full = s_full + 1;
+    uint64_t *acc_done = ds_full + 1;
+    uint64_t *mma_done = acc_done + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x;
+    const int t = p.kv_order[item / p.Hkvl];
+    const int kvh = item % p.Hkvl;
+    const int G = p.Hl / p.Hkvl;
+    const int qt0 = t;
+    const int n_q = static_cast<int>((p.kv_qend[t] + kTileM - 1) / kTileM) - qt0;
+    const int n_it = G * n_q;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(&qdo_full[s], 1);
+            mbar_init(&qdo_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(acc_done, 1);
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+    WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full, 2 * C::TILE_BYTES);
+            tma_tile<D>(&tmK, sK, kv_full, kvh, t * kTileN);
+            tma_tile<D>(&tmV, sV, kv_full, kvh, t * kTileN);
+            int last_use[C::NST];
+#pragma unroll
+            for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
+            for (int it = 0; it < n_it; ++it) {
+                const int s = it % C::NST, u = it / C::NST;
+                const int h = kvh * G + it / n_q;
+                const int qt = qt0 + it % n_q;
+                if (u > 0 && !mbar_wait(&qdo_empty[s], (u - 1) & 1, wc)) break;
+                mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES + 2 * 512);
+                tma_tile<D>(&tmQ, sQ + s * C::TILE_BYTES, &qdo_full[s], h, qt * kTileM);
+                tma_tile<D>(&tmDO, sDO + s * C::TILE_BYTES, &qdo_full[s], h, qt * kTileM);
+                const int64_t roff = static_cast<int64_t>(h) * p.Npad + static_cast<int64_t>(qt) * kTileM;
+                bulk_load(sRow + (s * 2 + 0) * 128, p.lse2 + roff, 512, &qdo_full[s]);
+                bulk_load(sRow + (s * 2 + 1) * 128, p.delta + roff, 512, &qdo_full[s]);
+                last_use[s] = u;
+            }
+            WaitCtx drain{p.wait_limit_ns, p.status, false};
+            mbar_wait(kv_full, 0, drain);
+            for (int s = 0; s < C::NST; ++s)
+                if (last_use[s] >= 0) mbar_wait(&qdo_full[s], last_use[s] & 1, drain);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
+            bool ok = mbar_wait(kv_full, 0, wc);
+            for (int it = 0; ok && it < n_it; ++it) {
+                const int s = it % C::NST, u = it / C::NST;
+                if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tbase + C::T_S, kmajor_desc<D>(aK, kk), kmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
+                            C::IDESC_SS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tbase + C::T_DP, kmajor_desc<D>(aV, kk), kmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
+                            C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_commit(s_full);
+                if (!mbar_wait(ds_full, it & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTileM / 16; ++kk) {
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    umma_ts(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
+                            C::IDESC_TS, acc);   // dV += P^T dO
+                    umma_ts(tbase + C::T_ACC1, tbase + C::T_DP + kk * 8, mnmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
+                            C::IDESC_TS, acc);   // dK += dS^T Q
+                }
+                umma_commit(&qdo_empty[s]);
+            }
+            if (ok) umma_commit(acc_done);
+            umma_commit(mma_done);
+            WaitCtx drain{p.wait_limit_ns, p.status, false};
+            mbar_wait(mma_done, 0, drain);
+        }
+    } else if (warp >= kComputeWarp0) {
+        // ------------------------------------------------ compute warpgroup: thread r owns key row r
+        const int r = threadIdx.x - kComputeWarp0 * 32;
+        const uint32_t lane_off = static_cast<uint32_t>((warp - kComputeWarp0) * 32) << 16;
+        const int j = t * kTileN + r;
+        // keys past N see no query; otherwise the queries of key j are [j, dend)
+        int dend = j;
+        if (j < p.N) {
+            int lo = j, hi = p.N;   // doc_start[lo] <= j; find the first index with doc_start > j
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (p.doc_start[mid] <= j) lo = mid; else hi = mid;
+            }
+            dend = hi;
+        }
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int s = it % C::NST, u = it / C::NST;
+            const int q0 = (qt0 + it % n_q) * kTileM;
+            if (!mbar_wait(s_full, it & 1, wc)) { ok = false; break; }
+            if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const float *rl = sRow + (s * 2 + 0) * 128;
+            const float *rd = sRow + (s * 2 + 1) * 128;
+            const bool need_mask = (q0 < j) || (q0 + kTileM - 1 >= dend);
+            const bool any_mask = __any_sync(0xffffffffu, need_mask);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sr[64], dr[64];
+                tmem_ld64(tbase + C::T_S + lane_off + half * 64, sr);
+                tmem_ld64(tbase + C::T_DP + lane_off + half * 64, dr);
+                tmem_ld_wait();
+                uint32_t pp[32], dd[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float pv[2], dv[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int c = half * 64 + 2 * e + k;
+                        float x = __uint_as_float(sr[2 * e + k]);
+                        if (any_mask) {
+                            const int qi = q0 + c;
+                            if (qi < j || qi >= dend) x = -CUDART_INF_F;
+                        }
+                        pv[k] = ex2_approx(fmaf(x, sl2, -rl[c]));
+                        dv[k] = pv[k] * (__uint_as_float(dr[2 * e + k]) - rd[c]);
+                    }
+                    pp[e] = pack_bf16x2(pv[0], pv[1]);
+                    dd[e] = pack_bf16x2(dv[0], dv[1]);
+                }
+                tmem_st32(tbase + C::T_S + lane_off + half * 32, pp);    // P^T  (queries packed in pairs)
+                tmem_st32(tbase + C::T_DP + lane_off + half * 32, dd);   // dS^T
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        if (ok && mbar_wait(acc_done, 0, wc)) {
+            tc_fence_after();
+            const bool valid = j < p.N;
+            __nv_bfloat16 *dv_row = p.dv + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D;
+            __nv_bfloat16 *dk_row = p.dk + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const float mul = which == 0 ? 1.f : p.scale;
+                __nv_bfloat16 *row = which == 0 ? dv_row : dk_row;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t raw[32];
+                    tmem_ld32(tbase + (which == 0 ? C::T_ACC0 : C::T_ACC1) + lane_off + c * 32, raw);
+                    tmem_ld_wait();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * mul, __uint_as_float(raw[2 * e + 1]) * mul);
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(row + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+}
+
+// ============================================================== dQ
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdParams p)
+{
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem + C::Q_OFF_Q;
+    uint8_t *sDO = smem + C::Q_OFF_DO;
+    uint8_t *sK = smem + C::Q_OFF_K;
+    uint8_t *sV = smem + C::Q_OFF_V;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::Q_OFF_BAR);
+    uint64_t *qdo_full = bars;
+    uint64_t *kv_full = bars + 1;           // [NST]
+    uint64_t *kv_empty = kv_full + C::NST;  // [NST]
+    uint64_t *s_full = kv_empty + C::NST;
+    uint64_t *ds_full = s_full + 1;
+    uint64_t *acc_done = ds_full + 1;
+    uint64_t *mma_done = acc_done + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x;
+    const int qt = p.q_order[item / p.Hl];
+    const int h = item % p.Hl;
+    const int kvh = h / (p.Hl / p.Hkvl);
+    const int kt0 = p.tile_lo[qt] / kTileN;
+    const int n_kv = qt - kt0 + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(qdo_full, 1);
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(acc_done, 1);
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+    WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(qdo_full, 2 * C::TILE_BYTES);
+            tma_tile<D>(&tmQ, sQ, qdo_full, h, qt * kTileM);
+            tma_tile<D>(&tmDO, sDO, qdo_full, h, qt * kTileM);
+            int last_use[C::NST];
+#pragma unroll
+            for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j % C::NST, u = j / C::NST;
+                if (u > 0 && !mbar_wait(&kv_empty[s], (u - 1) & 1, wc)) break;
+                mbar_arrive_expect_tx(&kv_full[s], 2 * C::TILE_BYTES);
+                tma_tile<D>(&tmK, sK + s * C::TILE_BYTES, &kv_full[s], kvh, (kt0 + j) * kTileN);
+                tma_tile<D>(&tmV, sV + s * C::TILE_BYTES, &kv_full[s], kvh, (kt0 + j) * kTileN);
+                last_use[s] = u;
+            }
+            WaitCtx drain{p.wait_limit_ns, p.status, false};
+            mbar_wait(qdo_full, 0, drain);
+            for (int s = 0; s < C::NST; ++s)
+                if (last_use[s] >= 0) mbar_wait(&kv_full[s], last_use[s] & 1, drain);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
+            bool ok = mbar_wait(qdo_full, 0, wc);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j % C::NST, u = j / C::NST;
+                if (!mbar_wait(&kv_full[s], u & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tbase + C::T_S, kmajor_desc<D>(aQ, kk), kmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
+                            C::IDESC_SS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tbase + C::T_DP, kmajor_desc<D>(aDO, kk), kmajor_desc<D>(aV + s * C::TILE_BYTES, kk),
+                            C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_commit(s_full);
+                if (!mbar_wait(ds_full, j & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk)
+                    umma_ts(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
+                            C::IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);   // dQ += dS K
+                umma_commit(&kv_empty[s]);
+            }
+            if (ok) umma_commit(acc_done);
+            umma_commit(mma_done);
+            WaitCtx drain{p.wait_limit_ns, p.status, false};
+            mbar_wait(mma_done, 0, drain);
+        }
+    } else if (warp >= kComputeWarp0) {
+        const int r = threadIdx.x - kComputeWarp0 * 32;
+        const uint32_t lane_off = static_cast<uint32_t>((warp - kComputeWarp0) * 32) << 16;
+        const int i = qt * kTileM + r;
+        const bool valid = i < p.N;
+        const int lo = valid ? p.doc_start[i] : i;
+        const float l2 = p.lse2[static_cast<int64_t>(h) * p.Npad + i];
+        const float di = p.delta[static_cast<int64_t>(h) * p.Npad + i];
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int c0 = (kt0 + j) * kTileN;
+            if (!mbar_wait(s_full, j & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const bool need_mask = (c0 < lo) || (c0 + kTileN - 1 > i);
+            const bool any_mask = __any_sync(0xffffffffu, need_mask);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sr[64], dr[64];
+                tmem_ld64(tbase + C::T_S + lane_off + half * 64, sr);
+                tmem_ld64(tbase + C::T_DP + lane_off + half * 64, dr);
+                tmem_ld_wait();
+                uint32_t dd[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float dv[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int c = half * 64 + 2 * e + k;
+                        float x = __uint_as_float(sr[2 * e + k]);
+                        if (any_mask) {
+                            const int key = c0 + c;
+                            if (key < lo || key > i) x = -CUDART_INF_F;
+                        }
+                        const float pv = ex2_approx(fmaf(x, sl2, -l2));
+                        dv[k] = pv * (__uint_as_float(dr[2 * e + k]) - di);
+                    }
+                    dd[e] = pack_bf16x2(dv[0], dv[1]);
+                }
+                tmem_st32(tbase + C::T_S + lane_off + half * 32, dd);   // dS (keys packed in pairs)
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        if (ok && mbar_wait(acc_done, 0, wc)) {
+            tc_fence_after();
+            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hl + h) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t raw[32];
+                tmem_ld32(tbase + C::T_ACC0 + lane_off + c * 32, raw);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * p.scale, __uint_as_float(raw[2 * e + 1]) * p.scale);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(row + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes, bool *done)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
+{
+    using C = BwdCfg<D>;
+    static_assert(C::KV_SMEM <= 232448 && C::Q_SMEM <= 232448, "shared memory budget");
+    const int T = static_cast<int>(ceil_div(a.N, kTileM));
+    const int Npad = T * kTileM;
+    alignas(64) CUtensorMap tq, tk, tv, tdo;
+    const int64_t qs = int64_t(a.Hl) * D * 2, ks = int64_t(a.Hkvl) * D * 2;
+    if (!encode_tmap_3d(&tq, a.q, D, a.Hl, a.N, int64_t(D) * 2, qs, C::AW, kTileM, C::SW) ||
+        !encode_tmap_3d(&tdo, a.dout, D, a.Hl, a.N, int64_t(D) * 2, qs, C::AW, kTileM, C::SW) ||
+        !encode_tmap_3d(&tk, a.k, D, a.Hkvl, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW) ||
+        !encode_tmap_3d(&tv, a.v, D, a.Hkvl, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW))
+        return cudaErrorInvalidValue;
+    BwdParams p;
+    p.doc_start = reinterpret_cast<const int32_t *>(a.ws + a.L.doc_start);
+    p.tile_lo = reinterpret_cast<const int32_t *>(a.ws + a.L.tile_lo);
+    p.q_order = reinterpret_cast<const int32_t *>(a.ws + a.L.q_order);
+    p.kv_qend = reinterpret_cast<const int32_t *>(a.ws + a.L.kv_qend);
+    p.kv_order = reinterpret_cast<const int32_t *>(a.ws + a.L.kv_order);
+    float *delta = reinterpret_cast<float *>(a.ws + a.L.delta);
+    float *lse2 = reinterpret_cast<float *>(a.ws + a.L.lse2);
+    p.delta = delta;
+    p.lse2 = lse2;
+    p.dq = static_cast<__nv_bfloat16 *>(a.dq);
+    p.dk = static_cast<__nv_bfloat16 *>(a.dk);
+    p.dv = static_cast<__nv_bfloat16 *>(a.dv);
+    p.N = static_cast<int>(a.N);
+    p.Npad = Npad;
+    p.T = T;
+    p.Hl = a.Hl;
+    p.Hkvl = a.Hkvl;
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * kLog2e;
+    p.status = reinterpret_cast<uint32_t *>(a.ws + a.L.status);
+    p.wait_limit_ns = a.wait_limit_ns;
+
+    const int64_t prep_threads = int64_t(a.Hl) * Npad * 32;
+    bwd_prep_kernel<D><<<static_cast<unsigned>(ceil_div(prep_threads, 256)), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, delta, lse2,
+        p.N, Npad, a.Hl);
+    static bool kv_attr[64] = {}, q_attr[64] = {};
+    cudaError_t e = set_smem(attn_bwd_dkdv_kernel<D>, C::KV_SMEM, kv_attr);
+    if (e != cudaSuccess) return e;
+    e = set_smem(attn_bwd_dq_kernel<D>, C::Q_SMEM, q_attr);
+    if (e != cudaSuccess) return e;
+    attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(int64_t(T) * a.Hkvl), kBwdThreads, C::KV_SMEM, stream>>>(
+        tq, tk, tv, tdo, p);
+    attn_bwd_dq_kernel<D><<<static_cast<unsigned>(int64_t(T) * a.Hl), kBwdThreads, C::Q_SMEM, stream>>>(
+        tq, tk, tv, tdo, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd(const BwdLaunch &a, cudaStream_t stream)
+{
+    switch (a.d) {
+    case 32: return launch_bwd_d<32>(a, stream);
+    case 64: return launch_bwd_d<64>(a, stream);
+    case 128: return launch_bwd_d<128>(a, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 }  // namespace uly

@@ -7,18 +7,25 @@
 // communication, because heads are independent. Work stays O(n^2) but memory is
 // O(n) by tiling with an online softmax (section "超长序列训练的挑战").
 //
-// One CTA computes one 128-row query tile of one head:
-//   warp 0      TMA producer: Q once, then K and V tiles into an NST-stage ring
-//   warp 1      allocates tensor memory; lane 0 issues every tcgen05.mma
-//   warps 4..7  softmax warpgroup: thread t owns query row t (TMEM lane t)
-// Tensor memory (512 columns): S double buffer at columns 0 and 128 (fp32
-// 128x128), O accumulator at column 256 (fp32 128 x d).
-// Per key tile j:  S_j = Q K_j^T (SS MMA, both K-major) -> softmax reads S_j,
-// masks diagonal / document-boundary tiles only, updates the running max with
-// lazy rescaling (O and l are rescaled only when the max grows by more than
-// 2^8), writes P_j = exp2(...) as bf16 into a 128B-swizzled shared buffer ->
-// O += P_j V_j (SS MMA, V read MN-major straight from its TMA tile).
-// Key tiles outside [doc_start(first row), last row] are never visited.
+// One CTA computes two consecutive 128-row query tiles A = 2u and B = 2u+1 of
+// one head; they share every K/V tile load.
+//   warps 0..3   softmax warpgroup of tile A (thread t owns row t = TMEM lane t)
+//   warps 4..7   softmax warpgroup of tile B
+//   warp 8       TMA producer: Q_A, Q_B, then K and V tiles into an NST-stage ring
+//   warp 9       allocates tensor memory; lane 0 issues every tcgen05.mma
+// Tensor memory (512 columns): S_A at 0, S_B at 128 (fp32 128x128 each; the
+// bf16 probabilities P overwrite the first 64 columns of their own S), O_A at
+// 256, O_B at 256 + d.
+// The issue order ping-pongs the two tiles so that one warpgroup's softmax runs
+// while the tensor core works on the other tile:
+//     ... PV_A(j-1), S_A(j), PV_B(j-1), S_B(j), PV_A(j), S_A(j+1) ...
+// S = Q K^T is an SS MMA (both operands K-major in 128B-swizzled shared memory);
+// O += P V is a TS MMA (P from tensor memory, V MN-major from its TMA tile).
+// The softmax reads its S row, masks only diagonal / document-boundary tiles,
+// keeps a running max with lazy rescaling (O and l are rescaled only when the
+// max grows by more than 2^8), and writes P = exp2(...) back as bf16.
+// Key tiles outside [doc_start(first row), last row] of a tile are never
+// visited by that tile.
 #include "ptx.cuh"
 #include "ulysses_internal.cuh"
 
@@ -29,9 +36,17 @@ namespace uly {
 
 namespace {
 
-constexpr int kFwdThreads = 256;
-constexpr int kSoftmaxWarp0 = 4;   // first warp of the softmax warpgroup
+constexpr int kFwdThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
+// Register split: launched at 168 per thread (384 x 168 = 64512); the two
+// softmax warpgroups take 224, the producer / MMA warpgroup keeps 56:
+// 256 x 224 + 128 x 56 = 64512.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kControlRegs = 72;
+static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= kFwdThreads * kLaunchRegs, "register split");
 
 struct FwdParams {
     const int32_t *doc_start;
@@ -41,7 +56,7 @@ struct FwdParams {
     int64_t o_row_elems;   // elements between consecutive token rows of O
     int o_head0;
     float *lse;
-    int N, Hl, Hkvl;
+    int N, T, Hl, Hkvl;
     int q_head0, kv_head0;
     float scale_log2;      // softmax scale * log2(e)
     uint32_t *status;
@@ -56,17 +71,18 @@ struct FwdCfg {
     static constexpr int ATOM_BYTES = kTileM * SW;            // one 128-row atom block
     static constexpr int TILE_BYTES = kTileM * D * 2;         // a Q, K or V tile
     static constexpr int NST = (D == 128) ? 2 : 4;            // K/V pipeline stages
-    static constexpr int P_BYTES = kTileM * kTileN * 2;       // one P buffer (two 128B atoms)
     static constexpr uint32_t SWZ = (SW == 128) ? kSwizzle128 : kSwizzle64;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = TILE_BYTES;
+    static constexpr int OFF_Q = 0;                           // Q_A, Q_B
+    static constexpr int OFF_K = 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
-    static constexpr int OFF_P = OFF_V + NST * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-    static constexpr int NBAR = 1 + 4 * NST + 8 + 1;
+    static constexpr int OFF_BAR = OFF_V + NST * TILE_BYTES;
+    static constexpr int NBAR = 2 + 4 * NST + 2 + 2 + 2 + 1;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kTileM, kTileN, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kTileM, D, false, true);
+    // tensor-memory columns: S / P of tile x at ts_col(x), O of tile x at to_col(x)
+    __host__ __device__ static constexpr uint32_t ts_col(int x) { return static_cast<uint32_t>(x) * 128u; }
+    __host__ __device__ static constexpr uint32_t to_col(int x) { return 256u + static_cast<uint32_t>(x * D); }
 };
 
 template <int D>
@@ -80,50 +96,53 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint8_t *sQ = smem + C::OFF_Q;
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
-    uint8_t *sP = smem + C::OFF_P;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *q_full = bars;
-    uint64_t *k_full = bars + 1;
+    uint64_t *q_full = bars;                 // [2]
+    uint64_t *k_full = bars + 2;             // [NST]
     uint64_t *k_empty = k_full + C::NST;
     uint64_t *v_full = k_empty + C::NST;
     uint64_t *v_empty = v_full + C::NST;
-    uint64_t *s_full = v_empty + C::NST;   // [2]
-    uint64_t *s_free = s_full + 2;         // [2]
-    uint64_t *p_full = s_free + 2;         // [2]
-    uint64_t *pv_done = p_full + 2;        // [2]
-    uint64_t *mma_done = pv_done + 2;
+    uint64_t *s_full = v_empty + C::NST;     // [2] per tile
+    uint64_t *p_full = s_full + 2;           // [2] per tile
+    uint64_t *o_done = p_full + 2;           // [2] per tile
+    uint64_t *mma_done = o_done + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work item: heaviest query tiles first
+    // ---- work item: a pair of query tiles, heaviest pairs first
     const int item = blockIdx.x;
-    const int tile = p.q_order[item / p.Hl];
+    const int pair = p.q_order[item / p.Hl];
     const int h = item % p.Hl;
     const int kvh = h / (p.Hl / p.Hkvl);
-    const int row0 = tile * kTileM;
-    const int kv_t0 = p.tile_lo[tile] / kTileN;
-    const int n_kv = tile - kv_t0 + 1;
+    const int tA = 2 * pair, tB = 2 * pair + 1;
+    const bool hasB = tB < p.T;
+    const int j0 = p.tile_lo[tA] / kTileN;                 // first key tile of the union
+    const int nA = tA - j0 + 1;                            // key tiles of A: union [0, nA)
+    const int loB = hasB ? p.tile_lo[tB] / kTileN : 0;
+    const int bstart = hasB ? loB - j0 : 0;                // key tiles of B: union [bstart, n_union)
+    const int nB = hasB ? tB - loB + 1 : 0;
+    const int n_union = hasB ? tB - j0 + 1 : nA;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        mbar_init(&q_full[0], 1);
+        mbar_init(&q_full[1], 1);
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&s_free[b], 128);
-            mbar_init(&p_full[b], 128);
-            mbar_init(&pv_done[b], 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 128);
+            mbar_init(&o_done[x], 1);
         }
         mbar_init(mma_done, 1);
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_holder, kTmemCols);
         tmem_relinquish();
     }
@@ -131,28 +150,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_holder;
-    const uint32_t tS = tbase;          // + b*128
-    const uint32_t tO = tbase + 256;
 
     // A CTA that starts after another one has timed out skips its work.
     WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
 
-    if (warp == 0) {
+    if (warp >= 8) {
+    setmaxnreg_dec<kControlRegs>();
+    if (warp == kProducerWarp) {
         // ================================================================ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+            for (int x = 0; x < (hasB ? 2 : 1); ++x) {
+                mbar_arrive_expect_tx(&q_full[x], C::TILE_BYTES);
 #pragma unroll
-            for (int a = 0; a < C::NA; ++a)
-                tma_load_3d(sQ + a * C::ATOM_BYTES, &tmQ, q_full, a * C::AW, p.q_head0 + h, row0);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_3d(sQ + x * C::TILE_BYTES + a * C::ATOM_BYTES, &tmQ, &q_full[x], a * C::AW,
+                                p.q_head0 + h, (x == 0 ? tA : tB) * kTileM);
+            }
             int last_k_use[C::NST], last_v_use[C::NST];
 #pragma unroll
             for (int s = 0; s < C::NST; ++s) last_k_use[s] = last_v_use[s] = -1;
-            for (int j = 0; j < n_kv; ++j) {
+            for (int j = 0; j < n_union; ++j) {
                 const int s = j % C::NST, u = j / C::NST;
-                const int key0 = (kv_t0 + j) * kTileN;
+                const int key0 = (j0 + j) * kTileN;
                 if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) break;
                 mbar_arrive_expect_tx(&k_full[s], C::TILE_BYTES);
 #pragma unroll
@@ -170,91 +192,116 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             // Never leave the CTA with bulk copies still landing in its shared memory.
             WaitCtx drain{p.wait_limit_ns, p.status, false};
-            mbar_wait(q_full, 0, drain);
+            mbar_wait(&q_full[0], 0, drain);
+            if (hasB) mbar_wait(&q_full[1], 0, drain);
             for (int s = 0; s < C::NST; ++s) {
                 if (last_k_use[s] >= 0) mbar_wait(&k_full[s], last_k_use[s] & 1, drain);
                 if (last_v_use[s] >= 0) mbar_wait(&v_full[s], last_v_use[s] & 1, drain);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-            auto issue_pv = [&](int jj) -> bool {
-                const int s = jj % C::NST, u = jj / C::NST, pb = jj & 1;
-                if (!mbar_wait(&v_full[s], u & 1, wc)) return false;
-                if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, wc)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk) {
-                    // A = P (128 rows x 128 keys, K-major, two 128B atoms of 64 keys)
-                    const uint64_t ad = smem_desc(aP + pb * C::P_BYTES + (kk >> 2) * (kTileM * 128) + (kk & 3) * 32,
-                                                  16, 1024, kSwizzle128);
-                    // B = V tile (keys x d), d contiguous: MN-major; 16 keys = 16 atom rows
-                    const uint64_t bd = smem_desc(aV + s * C::TILE_BYTES + kk * 16 * C::SW, C::ATOM_BYTES,
-                                                  8 * C::SW, C::SWZ);
-                    umma_ss(tO, ad, bd, C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&pv_done[pb]);
-                umma_commit(&v_empty[s]);
-                return true;
-            };
-            bool ok = mbar_wait(q_full, 0, wc);
-            int j = 0;
-            for (; ok && j < n_kv; ++j) {
-                const int s = j % C::NST, u = j / C::NST, b = j & 1;
-                if (!mbar_wait(&k_full[s], u & 1, wc)) { ok = false; break; }
-                if (j >= 2 && !mbar_wait(&s_free[b], ((j >> 1) - 1) & 1, wc)) { ok = false; break; }
-                tc_fence_after();
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            // S_x(it) = Q_x K_j^T, K-major operands, 16-element K steps
+            auto issue_s = [&](int x, int s) {
+                constexpr int steps = C::SW / 32;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    constexpr int steps = C::SW / 32;   // 16-element K steps per atom row
                     const uint32_t koff = (kk / steps) * C::ATOM_BYTES + (kk % steps) * 32;
-                    const uint64_t ad = smem_desc(aQ + koff, 16, 8 * C::SW, C::SWZ);
+                    const uint64_t ad = smem_desc(aQ + x * C::TILE_BYTES + koff, 16, 8 * C::SW, C::SWZ);
                     const uint64_t bd = smem_desc(aK + s * C::TILE_BYTES + koff, 16, 8 * C::SW, C::SWZ);
-                    umma_ss(tS + b * 128, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+                    umma_ss(tbase + C::ts_col(x), ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[b]);
-                umma_commit(&k_empty[s]);
-                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+                umma_commit(&s_full[x]);
+            };
+            // O_x += P_x V_j, P from tensor memory (8 columns per 16 keys)
+            auto issue_pv = [&](int x, int s, bool first) {
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk) {
+                    const uint64_t bd = smem_desc(aV + s * C::TILE_BYTES + kk * 16 * C::SW, C::ATOM_BYTES,
+                                                  8 * C::SW, C::SWZ);
+                    umma_ts(tbase + C::to_col(x), tbase + C::ts_col(x) + kk * 8, bd, C::IDESC_PV,
+                            (!first || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(&q_full[0], 0, wc);
+            if (ok && hasB) ok = mbar_wait(&q_full[1], 0, wc);
+            for (int j = 0; ok && j <= n_union; ++j) {
+                const int s = j % C::NST, u = j / C::NST;
+                const int sp = (j - 1 + C::NST) % C::NST, up = (j - 1) / C::NST;   // stage of key tile j-1
+                const bool have_j = j < n_union;
+                const bool pvA = (j - 1 >= 0) && (j - 1 < nA);
+                const bool sA = have_j && j < nA;
+                const int jb = j - bstart;
+                const bool pvB = hasB && (jb - 1 >= 0) && (jb - 1 < nB);
+                const bool sB = hasB && have_j && jb >= 0 && jb < nB;
+                if ((pvA || pvB) && !mbar_wait(&v_full[sp], up & 1, wc)) { ok = false; break; }
+                if ((sA || sB) && !mbar_wait(&k_full[s], u & 1, wc)) { ok = false; break; }
+                // tile A
+                if (pvA) {
+                    if (!mbar_wait(&p_full[0], (j - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(0, sp, j - 1 == 0);
+                    if (j - 1 == nA - 1) umma_commit(&o_done[0]);
+                }
+                if (sA) {
+                    tc_fence_after();
+                    issue_s(0, s);
+                }
+                // tile B
+                if (pvB) {
+                    if (!mbar_wait(&p_full[1], (jb - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(1, sp, jb - 1 == 0);
+                    if (jb - 1 == nB - 1) umma_commit(&o_done[1]);
+                }
+                if (sB) {
+                    tc_fence_after();
+                    issue_s(1, s);
+                }
+                if (sA || sB) umma_commit(&k_empty[s]);
+                if (pvA || pvB) umma_commit(&v_empty[sp]);
             }
-            if (ok) issue_pv(n_kv - 1);
             umma_commit(mma_done);
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(mma_done, 0, drain);
         }
-    } else if (warp >= kSoftmaxWarp0) {
-        // ================================================================ softmax warpgroup
-        const int r = threadIdx.x - kSoftmaxWarp0 * 32;           // query row within the tile == TMEM lane
-        const uint32_t lane_off = static_cast<uint32_t>((warp - kSoftmaxWarp0) * 32) << 16;
-        const int i = row0 + r;
+    }
+    } else {
+        setmaxnreg_inc<kSoftmaxRegs>();
+        // ================================================================ softmax warpgroups
+        const int x = warp >> 2;                                   // 0: tile A, 1: tile B
+        const int n_it = x == 0 ? nA : nB;
+        const int first_union = x == 0 ? 0 : bstart;
+        const int r = threadIdx.x & 127;                           // row within the tile == TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tbase + C::ts_col(x) + lane_off;
+        const uint32_t tO = tbase + C::to_col(x) + lane_off;
+        const int i = (x == 0 ? tA : tB) * kTileM + r;
         const bool valid = i < p.N;
         const int lo = valid ? p.doc_start[i] : i;
         const int hi = i;
         const float sl2 = p.scale_log2;
-        float ms = -CUDART_INF_F;   // running max actually used as exponent offset (scaled log2 units)
+        float ms = -CUDART_INF_F;   // exponent offset in use (scaled log2 units)
         float l = 0.f;
-        const uint32_t aP = smem_u32(sP);
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            const int b = j & 1;
-            if (!mbar_wait(&s_full[b], (j >> 1) & 1, wc)) { ok = false; break; }
+        for (int it = 0; it < n_it; ++it) {
+            if (!mbar_wait(&s_full[x], it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             float s[kTileN];
             {
-                uint32_t raw[32];
+                uint32_t raw0[64], raw1[64];
+                tmem_ld64(tS, raw0);
+                tmem_ld64(tS + 64, raw1);
+                tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < kTileN / 32; ++c) {
-                    tmem_ld32(tS + b * 128 + lane_off + c * 32, raw);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
+                for (int e = 0; e < 64; ++e) {
+                    s[e] = __uint_as_float(raw0[e]);
+                    s[64 + e] = __uint_as_float(raw1[e]);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&s_free[b]);
-
-            const int c0 = (kv_t0 + j) * kTileN;
+            const int c0 = (j0 + first_union + it) * kTileN;
             const bool need_mask = (c0 < lo) || (c0 + kTileN - 1 > hi);
             if (__any_sync(0xffffffffu, need_mask)) {
 #pragma unroll
@@ -263,9 +310,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     if (key < lo || key > hi) s[c] = -CUDART_INF_F;
                 }
             }
-            float mt = s[0];
+            float mx[8];
 #pragma unroll
-            for (int c = 1; c < kTileN; ++c) mt = fmaxf(mt, s[c]);
+            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < kTileN; c += 8)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
+            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             const float mt_s = mt * sl2;
             const bool resc = mt_s > ms + 8.0f;
             float alpha = 1.f;
@@ -274,47 +327,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 ms = mt_s;
                 l *= alpha;
             }
-            const float moff = (ms == -CUDART_INF_F) ? 0.f : ms;
-            uint32_t pk[kTileN / 2];
-            float lsum = 0.f;
-#pragma unroll
-            for (int c = 0; c < kTileN; c += 2) {
-                const float e0 = ex2_approx(fmaf(s[c], sl2, -moff));
-                const float e1 = ex2_approx(fmaf(s[c + 1], sl2, -moff));
-                lsum += e0 + e1;
-                pk[c / 2] = pack_bf16x2(e0, e1);
-            }
-            l += lsum;
-            // P buffer b was last read by PV_{j-2}
-            if (j >= 2 && !mbar_wait(&pv_done[b], ((j >> 1) - 1) & 1, wc)) { ok = false; break; }
-#pragma unroll
-            for (int q = 0; q < kTileN / 8; ++q) {
-                const uint32_t addr = aP + b * C::P_BYTES + (q >> 3) * (kTileM * 128) + r * 128 +
-                                      (((q & 7) ^ (r & 7)) << 4);
-                st_shared_v4(addr, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            }
-            fence_proxy_async_smem();
-            if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                // O holds sum_{j' < j} P_j' V_j' in the old units: rescale after PV_{j-1} lands
-                if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, wc)) { ok = false; break; }
-                tc_fence_after();
+            if (it > 0 && __any_sync(0xffffffffu, resc)) {
+                // O holds the previous tiles' sum in the old units. PV_x(it-1)
+                // was issued before S_x(it), so it has completed.
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t raw[32];
-                    tmem_ld32(tO + lane_off + c * 32, raw);
+                    tmem_ld32(tO + c * 32, raw);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-                    tmem_st32(tO + lane_off + c * 32, raw);
+                    tmem_st32(tO + c * 32, raw);
                 }
-                tmem_st_wait();
             }
+            const float moff = (ms == -CUDART_INF_F) ? 0.f : ms;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[64];
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+                const float e0 = ex2_approx(fmaf(s[2 * e], sl2, -moff));
+                const float e1 = ex2_approx(fmaf(s[2 * e + 1], sl2, -moff));
+                ls[(e & 1) * 2] += e0;
+                ls[(e & 1) * 2 + 1] += e1;
+                pk[e] = pack_bf16x2(e0, e1);
+            }
+            tmem_st64(tS, pk);   // P overwrites the first 64 columns of S
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&p_full[b]);
+            mbar_arrive(&p_full[x]);
         }
         // ---- epilogue: O / l -> bf16, LSE
-        const int last = n_kv - 1;
-        if (ok && mbar_wait(&pv_done[last & 1], (last >> 1) & 1, wc)) {
+        if (ok && n_it > 0 && mbar_wait(&o_done[x], 0, wc)) {
             tc_fence_after();
             const float inv_l = 1.f / l;
             __nv_bfloat16 *orow = p.o + static_cast<int64_t>(i) * p.o_row_elems +
@@ -322,7 +366,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t raw[32];
-                tmem_ld32(tO + lane_off + c * 32, raw);
+                tmem_ld32(tO + c * 32, raw);
                 tmem_ld_wait();
                 uint32_t w[16];
 #pragma unroll
@@ -341,7 +385,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+    if (warp == kMmaWarp) tmem_dealloc(tbase, kTmemCols);
 }
 
 template <int D>
@@ -367,6 +411,7 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.o_head0 = a.o_head0;
     p.lse = a.lse;
     p.N = static_cast<int>(a.N);
+    p.T = static_cast<int>(ceil_div(a.N, kTileM));
     p.Hl = a.Hl;
     p.Hkvl = a.Hkvl;
     p.q_head0 = a.q_head0;
@@ -383,8 +428,8 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const int64_t T = ceil_div(a.N, kTileM);
-    const int64_t items = T * a.Hl;
+    const int64_t pairs = ceil_div(p.T, 2);
+    const int64_t items = pairs * a.Hl;
     attn_fwd_kernel<D><<<static_cast<unsigned>(items), kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }

@@ -13,7 +13,8 @@
 // Kernels: a block-local scan, a fix-up with the carry of earlier blocks
 // (which also writes each query tile's first key), for the backward the last
 // query row of each key tile (a binary search over doc_start), and a counting
-// sort of tiles by work, heaviest first.
+// sort of the scheduling units (pairs of query tiles for the forward, key
+// tiles for the backward) by work, heaviest first.
 #include "ulysses_internal.cuh"
 
 namespace uly {
@@ -98,28 +99,42 @@ __global__ void kv_qend_kernel(int64_t N, int T, const int32_t *__restrict__ doc
     kv_qend[t] = static_cast<int32_t>(hi);
 }
 
-// Counting sort of T tiles by work, heaviest first. Work of query tile t is
-// the number of key tiles it visits; work of key tile t is the number of query
-// tiles that visit it. One CTA; hist lives in global scratch [T + 1].
-template <bool kKeyTiles>
-__global__ void __launch_bounds__(1024) tile_order_kernel(int T, const int32_t *__restrict__ src,
+// Work of one scheduling unit. kQueryPairs: unit u is the pair of query
+// tiles (2u, 2u+1), work = key tiles visited by both (src = tile_lo, each
+// query tile's first key). kQueryTiles: unit t is query tile t, work = key
+// tiles it visits. kKeyTiles: unit t is key tile t, work = query tiles that
+// visit it (src = kv_qend).
+enum class Unit { kQueryPairs, kQueryTiles, kKeyTiles };
+
+template <Unit kUnit>
+__device__ __forceinline__ int unit_work(int t, int T, const int32_t *__restrict__ src)
+{
+    if (kUnit == Unit::kKeyTiles) return static_cast<int>((src[t] + kTileM - 1) / kTileM) - t;
+    if (kUnit == Unit::kQueryTiles) return t - src[t] / kTileN + 1;
+    const int ta = 2 * t, tb = 2 * t + 1;
+    int w = ta - src[ta] / kTileN + 1;
+    if (tb < T) w += tb - src[tb] / kTileN + 1;
+    return w;
+}
+
+// Counting sort of `units` scheduling units by work (in [0, max_work]),
+// heaviest first. One CTA; hist lives in global scratch [max_work + 1].
+template <Unit kUnit>
+__global__ void __launch_bounds__(1024) unit_order_kernel(int units, int T, int max_work,
+                                                         const int32_t *__restrict__ src,
                                                          int32_t *__restrict__ hist, int32_t *__restrict__ order)
 {
     __shared__ int part[1024];
     const int tid = threadIdx.x;
-    for (int w = tid; w <= T; w += 1024) hist[w] = 0;
+    for (int w = tid; w <= max_work; w += 1024) hist[w] = 0;
     __syncthreads();
-    for (int t = tid; t < T; t += 1024) {
-        const int w = kKeyTiles ? (static_cast<int>((src[t] + kTileM - 1) / kTileM) - t)
-                                : (t - src[t] / kTileN + 1);
-        atomicAdd(&hist[w], 1);
-    }
+    for (int t = tid; t < units; t += 1024) atomicAdd(&hist[unit_work<kUnit>(t, T, src)], 1);
     __syncthreads();
-    // Exclusive prefix over work values in DESCENDING order:
-    // start[w] = number of tiles with work > w. Thread tid owns a contiguous
-    // segment of work values counted from the top.
-    const int per = (T + 1 + 1023) / 1024;
-    const int hi = T - tid * per;            // segment covers work values hi, hi-1, ..., hi-per+1
+    // Exclusive prefix over work values in DESCENDING order: the slot of the
+    // first unit with work w is the number of units with work > w. Thread tid
+    // owns a contiguous segment of work values counted from the top.
+    const int per = (max_work + 1 + 1023) / 1024;
+    const int hi = max_work - tid * per;     // segment covers work values hi, hi-1, ..., hi-per+1
     int sum = 0;
     for (int k = 0; k < per; ++k) {
         const int w = hi - k;
@@ -133,7 +148,7 @@ __global__ void __launch_bounds__(1024) tile_order_kernel(int T, const int32_t *
         part[tid] += add;
         __syncthreads();
     }
-    int run = part[tid] - sum;   // tiles with work above this segment
+    int run = part[tid] - sum;   // units with work above this segment
     for (int k = 0; k < per; ++k) {
         const int w = hi - k;
         if (w >= 0) {
@@ -143,10 +158,8 @@ __global__ void __launch_bounds__(1024) tile_order_kernel(int T, const int32_t *
         }
     }
     __syncthreads();
-    for (int t = tid; t < T; t += 1024) {
-        const int w = kKeyTiles ? (static_cast<int>((src[t] + kTileM - 1) / kTileM) - t)
-                                : (t - src[t] / kTileN + 1);
-        const int p = atomicAdd(&hist[w], 1);
+    for (int t = tid; t < units; t += 1024) {
+        const int p = atomicAdd(&hist[unit_work<kUnit>(t, T, src)], 1);
         order[p] = t;
     }
 }
@@ -165,14 +178,21 @@ cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLa
     doc_scan_kernel<<<nb, kScanBlock, 0, stream>>>(pos, N, doc_start, block_agg,
                                                    reinterpret_cast<uint32_t *>(ws + L.status));
     doc_fixup_kernel<<<nb, kScanBlock, 0, stream>>>(N, doc_start, block_agg, tile_lo);
-    tile_order_kernel<false><<<1, 1024, 0, stream>>>(static_cast<int>(T), tile_lo, scratch,
-                                                     reinterpret_cast<int32_t *>(ws + L.q_order));
-    if (backward) {
+    if (!backward) {
+        const int pairs = static_cast<int>(ceil_div(T, 2));
+        unit_order_kernel<Unit::kQueryPairs><<<1, 1024, 0, stream>>>(pairs, static_cast<int>(T),
+                                                                     static_cast<int>(2 * T), tile_lo, scratch,
+                                                                     reinterpret_cast<int32_t *>(ws + L.q_order));
+    } else {
+        unit_order_kernel<Unit::kQueryTiles><<<1, 1024, 0, stream>>>(static_cast<int>(T), static_cast<int>(T),
+                                                                     static_cast<int>(T), tile_lo, scratch,
+                                                                     reinterpret_cast<int32_t *>(ws + L.q_order));
         int32_t *kv_qend = reinterpret_cast<int32_t *>(ws + L.kv_qend);
         kv_qend_kernel<<<static_cast<int>(ceil_div(T, 256)), 256, 0, stream>>>(N, static_cast<int>(T), doc_start,
                                                                                kv_qend);
-        tile_order_kernel<true><<<1, 1024, 0, stream>>>(static_cast<int>(T), kv_qend, scratch,
-                                                        reinterpret_cast<int32_t *>(ws + L.kv_order));
+        unit_order_kernel<Unit::kKeyTiles><<<1, 1024, 0, stream>>>(static_cast<int>(T), static_cast<int>(T),
+                                                                   static_cast<int>(T), kv_qend, scratch,
+                                                                   reinterpret_cast<int32_t *>(ws + L.kv_order));
     }
     return cudaGetLastError();
 }

@@ -20,16 +20,18 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 //   status     uint32 [64]        status word (bit 0: a bounded wait ran out)
 //   doc_start  int32  [N]         first token of the row's document
 //   tile_lo    int32  [T]         doc_start of the first row of each 128-row tile
-//   q_order    int32  [T]         query tiles, heaviest first
+//   q_order    int32  [T]         forward: pairs of query tiles (2u, 2u+1), heaviest
+//                                 first; backward: single query tiles, heaviest first
 //   block_agg  int32  [ceil(N/1024)]  per-block maxima of the doc-start scan
-//   scratch    int32  [T + 1]     histogram for the tile sort
-// backward only:
+//   scratch    int32  [2T + 2]    histogram for the tile sort
+// backward only (Npad = T * 128):
 //   kv_qend    int32  [T]         one past the last row that attends to key tile t
 //   kv_order   int32  [T]         key tiles, heaviest first
-//   delta      fp32   [Hl][N]     D_i = sum_c dO_ic O_ic
+//   delta      fp32   [Hl][Npad]  D_i = sum_c dO_ic O_ic (0 on padding rows)
+//   lse2       fp32   [Hl][Npad]  LSE_i * log2(e) (+inf on padding rows)
 struct WsLayout {
     size_t status, doc_start, tile_lo, q_order, block_agg, scratch;
-    size_t kv_qend, kv_order, delta;
+    size_t kv_qend, kv_order, delta, lse2;
     size_t total;
 };
 
@@ -44,13 +46,14 @@ inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
     L.tile_lo = off;   off += align256(static_cast<size_t>(T) * 4);
     L.q_order = off;   off += align256(static_cast<size_t>(T) * 4);
     L.block_agg = off; off += align256(static_cast<size_t>(nb) * 4);
-    L.scratch = off;   off += align256(static_cast<size_t>(T + 1) * 4);
+    L.scratch = off;   off += align256(static_cast<size_t>(2 * T + 2) * 4);
     if (backward) {
         L.kv_qend = off;  off += align256(static_cast<size_t>(T) * 4);
         L.kv_order = off; off += align256(static_cast<size_t>(T) * 4);
-        L.delta = off;    off += align256(static_cast<size_t>(N) * Hl * 4);
+        L.delta = off;    off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
+        L.lse2 = off;     off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
     } else {
-        L.kv_qend = L.kv_order = L.delta = 0;
+        L.kv_qend = L.kv_order = L.delta = L.lse2 = 0;
     }
     L.total = off;
     return L;
@@ -60,8 +63,8 @@ inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
 cudaError_t launch_relayout(bool to_head, const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
                             cudaStream_t stream, int num_sms);
 
-// docbounds.cu: doc_start, tile_lo and the query-tile order (and, when
-// backward, kv_qend and the key-tile order).
+// docbounds.cu: doc_start, tile_lo and the query order (pairs of tiles for the
+// forward; single tiles, kv_qend and the key-tile order for the backward).
 cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
                              cudaStream_t stream);   // also clears the status word
 

@@ -8,6 +8,13 @@ import torch
 # max-abs 2e-2 and mean-abs 2e-3 (bf16 inputs, fp32 accumulation, bf16 O).
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
+# Gradients are stored in bf16 and can be larger than the forward's outputs:
+# rounding a value to bf16 alone moves it by up to 2^-9 of its magnitude (so a
+# flat 2e-2 cannot hold once |value| >= 8), and the bf16 P / dS operands of the
+# tensor-core products add up to 2^-9 of each term. For dQ, dK and dV the
+# per-element bound is therefore 2e-2 + 2^-8 * |ref| (two such roundings), with
+# the same mean-abs 2e-3.
+GRAD_REL = 2.0 ** -8
 
 
 def sample_rows(lengths, N: int, n_random: int, seed: int, cap_doc_edges: int = 64) -> np.ndarray:
@@ -37,9 +44,23 @@ def err_stats(got: np.ndarray, ref: np.ndarray):
     return float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0
 
 
-def assert_close(name: str, got: np.ndarray, ref: np.ndarray, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+def assert_close(name: str, got: np.ndarray, ref: np.ndarray, max_abs=MAX_ABS, mean_abs=MEAN_ABS, rel=0.0):
+    """Every element within max_abs + rel*|ref| of the reference, and the mean
+    absolute error within mean_abs."""
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    diff = np.abs(got.astype(np.float64) - ref)
     mx, mn = err_stats(got, ref)
-    assert mx <= max_abs and mn <= mean_abs, f"{name}: max-abs {mx:.3e} (<= {max_abs}), mean-abs {mn:.3e} (<= {mean_abs})"
+    excess = diff - rel * np.abs(ref)
+    k = int(np.argmax(excess)) if excess.size else 0
+    worst = float(excess.reshape(-1)[k]) if excess.size else 0.0
+    where = np.unravel_index(k, got.shape) if excess.size else ()
+    assert worst <= max_abs and mn <= mean_abs, (
+        f"{name}: worst |err| - {rel:g}|ref| = {worst:.3e} at {tuple(int(x) for x in where)} "
+        f"(ref {float(ref[where]) if excess.size else 0:.4f}, got {float(got[where]) if excess.size else 0:.4f}; "
+        f"limit {max_abs}), max-abs {mx:.3e}, mean-abs {mn:.3e} (<= {mean_abs})")
     return mx, mn
+
+
+def assert_grad_close(name: str, got: np.ndarray, ref: np.ndarray):
+    return assert_close(name, got, ref, rel=GRAD_REL)
