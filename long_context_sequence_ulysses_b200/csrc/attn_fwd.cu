@@ -23,7 +23,8 @@
 // O += P V is a TS MMA (P from tensor memory, V MN-major from its TMA tile).
 // The softmax reads its S row, masks only diagonal / document-boundary tiles,
 // keeps a running max with lazy rescaling (O and l are rescaled only when the
-// max grows by more than 2^8), and writes P = exp2(...) back as bf16.
+// max grows by more than 2^8), and writes P = exp2(...) back as bf16. The
+// row arithmetic uses the packed fp32x2 FMA / add and the 3-input max.
 // Key tiles outside [doc_start(first row), last row] of a tile are never
 // visited by that tile.
 #include "ptx.cuh"
@@ -201,7 +202,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ================================================================ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the loop; one elected lane issues each tcgen05
+        // instruction (faster than issuing from a one-lane branch).
+        {
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
             // S_x(it) = Q_x K_j^T, K-major operands, 16-element K steps
             auto issue_s = [&](int x, int s) {
@@ -211,9 +214,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const uint32_t koff = (kk / steps) * C::ATOM_BYTES + (kk % steps) * 32;
                     const uint64_t ad = smem_desc(aQ + x * C::TILE_BYTES + koff, 16, 8 * C::SW, C::SWZ);
                     const uint64_t bd = smem_desc(aK + s * C::TILE_BYTES + koff, 16, 8 * C::SW, C::SWZ);
-                    umma_ss(tbase + C::ts_col(x), ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+                    umma_ss_elect(tbase + C::ts_col(x), ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[x]);
+                umma_commit_elect(&s_full[x]);
             };
             // O_x += P_x V_j, P from tensor memory (8 columns per 16 keys)
             auto issue_pv = [&](int x, int s, bool first) {
@@ -221,12 +224,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int kk = 0; kk < kTileN / 16; ++kk) {
                     const uint64_t bd = smem_desc(aV + s * C::TILE_BYTES + kk * 16 * C::SW, C::ATOM_BYTES,
                                                   8 * C::SW, C::SWZ);
-                    umma_ts(tbase + C::to_col(x), tbase + C::ts_col(x) + kk * 8, bd, C::IDESC_PV,
-                            (!first || kk > 0) ? 1u : 0u);
+                    umma_ts_elect(tbase + C::to_col(x), tbase + C::ts_col(x) + kk * 8, bd, C::IDESC_PV,
+                                  (!first || kk > 0) ? 1u : 0u);
                 }
             };
-            bool ok = mbar_wait(&q_full[0], 0, wc);
-            if (ok && hasB) ok = mbar_wait(&q_full[1], 0, wc);
+            bool ok = mbar_wait_warp(&q_full[0], 0, wc);
+            if (ok && hasB) ok = mbar_wait_warp(&q_full[1], 0, wc);
             for (int j = 0; ok && j <= n_union; ++j) {
                 const int s = j % C::NST, u = j / C::NST;
                 const int sp = (j - 1 + C::NST) % C::NST, up = (j - 1) / C::NST;   // stage of key tile j-1
@@ -236,14 +239,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const int jb = j - bstart;
                 const bool pvB = hasB && (jb - 1 >= 0) && (jb - 1 < nB);
                 const bool sB = hasB && have_j && jb >= 0 && jb < nB;
-                if ((pvA || pvB) && !mbar_wait(&v_full[sp], up & 1, wc)) { ok = false; break; }
-                if ((sA || sB) && !mbar_wait(&k_full[s], u & 1, wc)) { ok = false; break; }
+                if ((pvA || pvB) && !mbar_wait_warp(&v_full[sp], up & 1, wc)) { ok = false; break; }
+                if ((sA || sB) && !mbar_wait_warp(&k_full[s], u & 1, wc)) { ok = false; break; }
                 // tile A
                 if (pvA) {
-                    if (!mbar_wait(&p_full[0], (j - 1) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait_warp(&p_full[0], (j - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(0, sp, j - 1 == 0);
-                    if (j - 1 == nA - 1) umma_commit(&o_done[0]);
+                    if (j - 1 == nA - 1) umma_commit_elect(&o_done[0]);
                 }
                 if (sA) {
                     tc_fence_after();
@@ -251,19 +254,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 // tile B
                 if (pvB) {
-                    if (!mbar_wait(&p_full[1], (jb - 1) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait_warp(&p_full[1], (jb - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(1, sp, jb - 1 == 0);
-                    if (jb - 1 == nB - 1) umma_commit(&o_done[1]);
+                    if (jb - 1 == nB - 1) umma_commit_elect(&o_done[1]);
                 }
                 if (sB) {
                     tc_fence_after();
                     issue_s(1, s);
                 }
-                if (sA || sB) umma_commit(&k_empty[s]);
-                if (pvA || pvB) umma_commit(&v_empty[sp]);
+                if (sA || sB) umma_commit_elect(&k_empty[s]);
+                if (pvA || pvB) umma_commit_elect(&v_empty[sp]);
             }
-            umma_commit(mma_done);
+            umma_commit_elect(mma_done);
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(mma_done, 0, drain);
         }
@@ -310,15 +313,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     if (key < lo || key > hi) s[c] = -CUDART_INF_F;
                 }
             }
-            float mx[8];
+            // row max: 4 independent chains of 3-input max
+            float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+            for (int c = 4; c < kTileN; c += 8)
 #pragma unroll
-            for (int c = 8; c < kTileN; c += 8)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[c + e]);
-            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[c + e], s[c + 4 + e]);
+            const float mt = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
             const float mt_s = mt * sl2;
             const bool resc = mt_s > ms + 8.0f;
             float alpha = 1.f;
@@ -341,18 +342,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
             }
             const float moff = (ms == -CUDART_INF_F) ? 0.f : ms;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // P = exp2(s * scale*log2(e) - offset): the argument two columns at a
+            // time (packed FMA), the exponential on the SFU, the row sum two
+            // columns at a time (packed add, 4 independent accumulator pairs).
+            float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[64];
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-                const float e0 = ex2_approx(fmaf(s[2 * e], sl2, -moff));
-                const float e1 = ex2_approx(fmaf(s[2 * e + 1], sl2, -moff));
-                ls[(e & 1) * 2] += e0;
-                ls[(e & 1) * 2 + 1] += e1;
+                float x0, x1;
+                fma2_bcast(x0, x1, s[2 * e], s[2 * e + 1], sl2, -moff);
+                const float e0 = ex2_approx(x0);
+                const float e1 = ex2_approx(x1);
+                add2_acc(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], e0, e1);
                 pk[e] = pack_bf16x2(e0, e1);
             }
             tmem_st64(tS, pk);   // P overwrites the first 64 columns of S
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_full[x]);

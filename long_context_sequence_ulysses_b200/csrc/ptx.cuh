@@ -48,12 +48,29 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+// Potentially blocking probe: the thread may sleep up to about `hint_ns`
+// (a suspend-time hint) waiting for the phase before returning false, so a
+// waiting warp does not take issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns = 20000u)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking probe: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -81,7 +98,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
     uint32_t spins = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (((++spins) & 63u) == 0u) {
+        if (((++spins) & 7u) == 0u) {
             // Give up when the deadline passes, or as soon as any CTA of the
             // grid has recorded a timeout (the launch has failed anyway).
             const bool other_failed = w.status && (*reinterpret_cast<volatile uint32_t *>(w.status) != 0u);
@@ -92,6 +109,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
             }
         }
     }
+}
+
+// Warp-uniform wait for warps whose lanes then execute elect.sync together:
+// either every lane sees success or every lane records failure.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, WaitCtx &w)
+{
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
+    if (!ok) w.failed = true;
+    return ok;
 }
 
 // ---------------------------------------------------------------- TMA
@@ -178,6 +204,43 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Warp-collective forms: every lane of a converged warp executes them and
+// elect.sync picks one lane (always the same one, the lowest active lane) to
+// issue the instruction.
+__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_elect(uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(smem_u32(bar))
         : "memory");
 }
 
@@ -283,6 +346,59 @@ __device__ __forceinline__ float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA / integer pipes, leaving the special-function unit free.
+// Range reduction 2^x = 2^j 2^f with j = round(x), f in [-1/2, 1/2] (Cody and
+// Waite); 2^f is the degree-3 minimax polynomial in relative error fitted by
+// long_context_sequence_ulysses_b200/exp2_poly.py (max relative error
+// 7.5e-5, far below the 2^-9 of the bf16 probabilities it feeds); 2^j is
+// added into the exponent field. x is clamped at -125 so that the result stays
+// a normal float; there it is ~2^-125 instead of 0, which no sum can see.
+__device__ __forceinline__ float ex2_poly(float x)
+{
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;          // 1.5 * 2^23: round(x) lands in the low mantissa bits
+    const float f = x - (t - 12582912.0f);
+    float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+    p = fmaf(p, f, 0.6932609677314758f);
+    p = fmaf(p, f, 0.9999280571937561f);
+    const int j = __float_as_int(t) - 0x4B400000;
+    return __int_as_float(__float_as_int(p) + (j << 23));
+}
+
+// Packed fp32 pair arithmetic (two lanes per instruction, IEEE round to
+// nearest): (d0, d1) = (a0, a1) * b + c with b and c broadcast.
+__device__ __forceinline__ void fma2_bcast(float &d0, float &d1, float a0, float a1, float b, float c)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%5, %5};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (d0, d1) += (a0, a1)
+__device__ __forceinline__ void add2_acc(float &d0, float &d1, float a0, float a1)
+{
+    asm("{\n\t.reg .b64 ra, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rd, {%0, %1};\n\t"
+        "add.rn.f32x2 rd, rd, ra;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1));
+}
+
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

@@ -1,0 +1,91 @@
+"""Ulysses across G GPUs: one process per GPU, torch.distributed over NCCL.
+
+Page "Hugging Face并行加速：10倍提升超长序列训练效率", section "Ulysses的工作原理":
+GPU g holds tokens [g*N/G, (g+1)*N/G) (step 序列分片); an all-to-all gives every
+GPU the whole sequence for H/G heads (step 全体间通信); attention runs locally
+(本地注意力计算); a second all-to-all restores sequence shards (全体间通信复原).
+
+The single-GPU relayout kernels are exactly the local halves of the exchange:
+  pack    ulysses_seq_to_head(shard [N/G][H][d], N/G, P=G) -> [G][N/G][H/G][d],
+          block r is what GPU r receives;
+  all_to_all_single(recv, send) then leaves [G src][N/G][H/G][d] = [N][H/G][d],
+          the head slice, with no unpacking;
+  unpack  ulysses_head_to_seq(recv [G][N/G][H/G][d], N/G, P=G) -> [N/G][H][d]
+          after the second exchange.
+The exchange moves raw bytes (tensors are sent as uint8 views), so it is
+dtype-agnostic and works on any backend that has all_to_all.
+
+The local steps are parameters (defaulting to the CUDA library) so that the
+host logic can be exercised with CPU stand-ins over gloo.
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional, Tuple
+
+import torch
+import torch.distributed as dist
+
+
+def _world(group) -> Tuple[int, int]:
+    return dist.get_world_size(group), dist.get_rank(group)
+
+
+def _cuda_pack(x: torch.Tensor, G: int) -> torch.Tensor:
+    import long_context_sequence_ulysses_b200 as U
+    return U.seq_to_head(x, G)
+
+
+def _cuda_unpack(y: torch.Tensor, G: int) -> torch.Tensor:
+    import long_context_sequence_ulysses_b200 as U
+    return U.head_to_seq(y, G)
+
+
+def seq_to_head(x_local: torch.Tensor, group=None,
+                pack: Optional[Callable[[torch.Tensor, int], torch.Tensor]] = None) -> torch.Tensor:
+    """[N/G][Hx][d] sequence shard -> [N][Hx/G][d] head slice of this rank."""
+    G, _ = _world(group)
+    n_loc, Hx, d = x_local.shape
+    if Hx % G or n_loc % G:
+        raise ValueError(f"heads ({Hx}) and local tokens ({n_loc}) must be divisible by the group size {G}")
+    send = (pack or _cuda_pack)(x_local, G)                     # [G][N/G][Hx/G][d]
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv.view(torch.uint8), send.contiguous().view(torch.uint8), group=group)
+    return recv.view(G * n_loc, Hx // G, d)
+
+
+def head_to_seq(y: torch.Tensor, group=None,
+                unpack: Optional[Callable[[torch.Tensor, int], torch.Tensor]] = None) -> torch.Tensor:
+    """[N][Hx/G][d] head slice -> [N/G][Hx][d] sequence shard of this rank."""
+    G, _ = _world(group)
+    N, Hl, d = y.shape
+    if N % G:
+        raise ValueError(f"N ({N}) must be divisible by the group size {G}")
+    send = y.contiguous().view(G, N // G, Hl, d)                # block r goes to rank r
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv.view(torch.uint8), send.view(torch.uint8), group=group)
+    return (unpack or _cuda_unpack)(recv, G)                     # [N/G][Hx][d]
+
+
+def gather_position_ids(pos_local: torch.Tensor, group=None) -> torch.Tensor:
+    """All ranks' position ids, in sequence order (each rank needs the whole
+    sequence's document structure once it holds whole-sequence head slices)."""
+    G, _ = _world(group)
+    parts = [torch.empty_like(pos_local) for _ in range(G)]
+    dist.all_gather(parts, pos_local.contiguous(), group=group)
+    return torch.cat(parts)
+
+
+def attention_forward(q_local: torch.Tensor, k_local: torch.Tensor, v_local: torch.Tensor,
+                      pos_local: torch.Tensor, group=None, scale: Optional[float] = None,
+                      attn: Optional[Callable] = None, pack=None, unpack=None):
+    """The Ulysses attention step of one rank: returns (o_local [N/G][H][d],
+    lse [H/G][N] for this rank's heads, position ids of the whole sequence)."""
+    pos = gather_position_ids(pos_local, group)
+    q = seq_to_head(q_local, group, pack)
+    k = seq_to_head(k_local, group, pack)
+    v = seq_to_head(v_local, group, pack)
+    if attn is None:
+        import long_context_sequence_ulysses_b200 as U
+        attn = U.attn_fwd
+    o, lse = attn(q, k, v, pos, scale=scale)
+    return head_to_seq(o, group, unpack), lse, pos

@@ -1,0 +1,59 @@
+"""Worker for the multi-process (gloo, CPU) tests of the Ulysses exchange.
+
+Each process holds one sequence shard, runs the library's exchange logic
+(long_context_sequence_ulysses_b200.dist) with CPU stand-ins for the local
+steps — the oracle's relayouts as pack/unpack and the oracle's attention —
+and returns its shard of O and LSE through a queue."""
+import os
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+
+def _bits_to_bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+def worker(rank: int, world: int, port: int, case: dict, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        _run(rank, world, case, out_q)
+    except Exception as e:  # report instead of leaving the parent waiting
+        out_q.put((rank, "error", repr(e), None))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(rank, world, case, out_q):
+    if True:
+        import oracle
+        from long_context_sequence_ulysses_b200 import dist as udist
+        from workloads import random_case
+
+        c = random_case(case["N"], case["H"], case["Hkv"], case["d"], case["lengths"], seed=case["seed"])
+        N, d = case["N"], case["d"]
+        n_loc = N // world
+        sl = slice(rank * n_loc, (rank + 1) * n_loc)
+
+        def pack(x, G):
+            n, Hx, dd = x.shape
+            return _bits_to_bf16(oracle.seq_to_head(x, n, G, Hx, dd))
+
+        def unpack(y, G):
+            Gp, n, Hl, dd = y.shape
+            return _bits_to_bf16(oracle.head_to_seq(y, n, G, Hl * G, dd)).view(n, Hl * G, dd)
+
+        def attn(q, k, v, pos, scale=None):
+            o, lse = oracle.attn_fwd(q, k, v, pos, scale=scale)
+            return torch.from_numpy(o).to(torch.bfloat16), torch.from_numpy(lse)
+
+        o_loc, lse, pos = udist.attention_forward(c["q"][sl].contiguous(), c["k"][sl].contiguous(),
+                                                  c["v"][sl].contiguous(), c["position_ids"][sl].contiguous(),
+                                                  attn=attn, pack=pack, unpack=unpack)
+        out_q.put((rank, o_loc.view(torch.int16).numpy().copy(), lse.numpy().copy(), pos.numpy().copy()))
+        dist.barrier()

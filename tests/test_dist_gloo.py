@@ -1,0 +1,54 @@
+"""The multi-GPU Ulysses exchange (long_context_sequence_ulysses_b200.dist),
+run as world_size 2 and 4 gloo processes on the CPU with the oracle standing
+in for the local kernels: the sharded result must equal the unsharded
+oracle's attention bit for bit (after the same bf16 rounding), since the
+exchange only moves data and heads are independent."""
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import oracle
+from workloads import random_case
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_exchange_matches_unsharded(world):
+    import dist_worker
+    case = {"N": 64, "H": 8, "Hkv": 4, "d": 32, "lengths": [23, 1, 40], "seed": 12}
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=dist_worker.worker, args=(r, world, port, case, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {}
+    try:
+        for _ in range(world):
+            r, o, lse, pos = q.get(timeout=90)
+            assert not (isinstance(o, str) and o == "error"), f"rank {r}: {lse}"
+            results[r] = (o, lse, pos)
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    c = random_case(case["N"], case["H"], case["Hkv"], case["d"], case["lengths"], seed=case["seed"])
+    ref_o, ref_lse = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    ref_bits = torch.from_numpy(ref_o).to(torch.bfloat16).view(torch.int16).numpy()
+    n_loc = case["N"] // world
+    Hl = case["H"] // world
+    for r in range(world):
+        o, lse, pos = results[r]
+        assert np.array_equal(o, ref_bits[r * n_loc:(r + 1) * n_loc])          # this rank's sequence shard
+        assert np.array_equal(lse, ref_lse[r * Hl:(r + 1) * Hl])               # this rank's heads
+        assert np.array_equal(pos, c["position_ids"].numpy())
