@@ -147,6 +147,116 @@ def workload_work(w, lengths):
 
 # --------------------------------------------------------------------------- GPU arm
 
+class Timer:
+    """CUDA events around one kind of launch, on the launching stream."""
+
+    def __init__(self, stream, enabled: bool):
+        self.stream = stream
+        self.enabled = enabled
+        self.ev = {"attn_fwd": [], "attn_bwd": [], "relayout": [], "exchange": []}
+
+    def __call__(self, kind, fn):
+        if not self.enabled:
+            return fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        r = fn()
+        b.record(self.stream)
+        self.ev[kind].append((a, b))
+        return r
+
+    def stats(self, kind):
+        xs = [a.elapsed_time(b) for a, b in self.ev[kind]]
+        return ((sum(xs) / len(xs)) if xs else None), (sum(xs) if xs else None)
+
+
+def build_single(U, w, inp, dev, timed):
+    """One GPU: the P ranks are emulated as P buffers, the exchanges are the
+    relayout kernels. Returns (step, our kernel launches per step, workspace)."""
+    P, N, d, Hl, Hkvl = w.P, w.N, w.d, w.Hl, w.Hkvl
+    pos = inp["position_ids"]
+    q_seq, k_seq, v_seq, do_seq = inp["q"], inp["k"], inp["v"], inp.get("do")
+    q_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
+    k_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    o_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
+    lse_all = torch.empty((P * Hl, N), dtype=torch.float32, device=dev)
+    o_seq = torch.empty_like(q_seq)
+    ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
+    if w.backward:
+        do_all = torch.empty_like(q_all)
+        dq_all, dk_all, dv_all = torch.empty_like(q_all), torch.empty_like(k_all), torch.empty_like(v_all)
+        dq_seq, dk_seq, dv_seq = torch.empty_like(q_seq), torch.empty_like(k_seq), torch.empty_like(v_seq)
+
+    def step():
+        # first all-to-all: every rank's head slice of Q, K, V
+        timed("relayout", lambda: U.seq_to_head(q_seq, P, out=q_all))
+        timed("relayout", lambda: U.seq_to_head(k_seq, P, out=k_all))
+        timed("relayout", lambda: U.seq_to_head(v_seq, P, out=v_all))
+        for r in range(P):
+            timed("attn_fwd", lambda: U.attn_fwd(q_all[r], k_all[r], v_all[r], pos, out=o_all[r],
+                                                 lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws))
+        if w.backward:
+            timed("relayout", lambda: U.seq_to_head(do_seq, P, out=do_all))
+            for r in range(P):
+                timed("attn_bwd", lambda: U.attn_bwd(q_all[r], k_all[r], v_all[r], o_all[r], do_all[r],
+                                                     lse_all[r * Hl:(r + 1) * Hl], pos, ws=ws, dq=dq_all[r],
+                                                     dk=dk_all[r], dv=dv_all[r]))
+            timed("relayout", lambda: U.head_to_seq(dq_all, P, out=dq_seq))
+            timed("relayout", lambda: U.head_to_seq(dk_all, P, out=dk_seq))
+            timed("relayout", lambda: U.head_to_seq(dv_all, P, out=dv_seq))
+        # second all-to-all: O back to sequence shards
+        timed("relayout", lambda: U.head_to_seq(o_all, P, out=o_seq))
+
+    launches = 3 + 4 * P + 1 + ((1 + BWD_LAUNCHES * P + 3) if w.backward else 0)
+    return step, launches, ws
+
+
+def build_multi(U, w, inp, dev, timed, G, rank):
+    """G GPUs: Ulysses with P = G real ranks. Each GPU holds tokens
+    [rank*N/G, (rank+1)*N/G); the pack before and the unpack after each NCCL
+    all-to-all are the relayout kernels; each GPU computes H/G heads."""
+    from long_context_sequence_ulysses_b200 import dist as udist
+    N, d = w.N, w.d
+    if w.H % G or w.Hkv % G or N % (G * G):
+        raise SystemExit(f"workload {w.name} cannot be split over {G} GPUs")
+    n_loc, Hg, Hkvg = N // G, w.H // G, w.Hkv // G
+    sl = slice(rank * n_loc, (rank + 1) * n_loc)
+    q_loc, k_loc, v_loc = (inp[x][sl].contiguous() for x in ("q", "k", "v"))
+    do_loc = inp["do"][sl].contiguous() if w.backward else None
+    pos_loc = inp["position_ids"][sl].contiguous()
+    buf = lambda h: torch.empty((G, n_loc, h, d), dtype=torch.bfloat16, device=dev)
+    sq, rq, sk, rk, sv, rv = buf(Hg), buf(Hg), buf(Hkvg), buf(Hkvg), buf(Hkvg), buf(Hkvg)
+    o_head, ro = torch.empty((N, Hg, d), dtype=torch.bfloat16, device=dev), buf(Hg)
+    o_loc = torch.empty_like(q_loc)
+    lse = torch.empty((Hg, N), dtype=torch.float32, device=dev)
+    pos = torch.empty(N, dtype=torch.int32, device=dev)
+    ws = torch.empty(U.workspace_bytes(N, Hg, Hkvg, d, w.backward), dtype=torch.uint8, device=dev)
+    if w.backward:
+        sdo, rdo = buf(Hg), buf(Hg)
+        dq_h, dk_h, dv_h = (torch.empty((N, h, d), dtype=torch.bfloat16, device=dev) for h in (Hg, Hkvg, Hkvg))
+        rdq, rdk, rdv = buf(Hg), buf(Hkvg), buf(Hkvg)
+        dq_loc, dk_loc, dv_loc = torch.empty_like(q_loc), torch.empty_like(k_loc), torch.empty_like(v_loc)
+
+    def step():
+        udist.gather_position_ids(pos_loc, out=pos)
+        q = timed("exchange", lambda: udist.seq_to_head(q_loc, send=sq, recv=rq))
+        k = timed("exchange", lambda: udist.seq_to_head(k_loc, send=sk, recv=rk))
+        v = timed("exchange", lambda: udist.seq_to_head(v_loc, send=sv, recv=rv))
+        timed("attn_fwd", lambda: U.attn_fwd(q, k, v, pos, out=o_head, lse=lse, ws=ws))
+        if w.backward:
+            g = timed("exchange", lambda: udist.seq_to_head(do_loc, send=sdo, recv=rdo))
+            timed("attn_bwd", lambda: U.attn_bwd(q, k, v, o_head, g, lse, pos, ws=ws, dq=dq_h, dk=dk_h, dv=dv_h))
+            timed("exchange", lambda: udist.head_to_seq(dq_h, recv=rdq, out=dq_loc))
+            timed("exchange", lambda: udist.head_to_seq(dk_h, recv=rdk, out=dk_loc))
+            timed("exchange", lambda: udist.head_to_seq(dv_h, recv=rdv, out=dv_loc))
+        timed("exchange", lambda: udist.head_to_seq(o_head, recv=ro, out=o_loc))
+
+    launches = 3 + 4 + 1 + ((1 + BWD_LAUNCHES + 3) if w.backward else 0)
+    return step, launches, ws
+
+
 def run_gpu(args):
     import long_context_sequence_ulysses_b200 as U
 
@@ -162,79 +272,25 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     w = WORKLOADS[args.workload]
-    P = w.P
     inp = make_inputs(w, device=dev)
-    pos = inp["position_ids"]
     lengths = inp["lengths"]
-    q_seq, k_seq, v_seq = inp["q"], inp["k"], inp["v"]
-    do_seq = inp.get("do")
-    Hl, Hkvl, d, N = w.Hl, w.Hkvl, w.d, w.N
     pairs, fwd_flop, bwd_flop, relayout_bytes = workload_work(w, lengths)
-
-    # head-slice buffers of all emulated ranks: [P][N][H/P][d]
-    q_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
-    k_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
-    v_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
-    o_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
-    lse_all = torch.empty((P * Hl, N), dtype=torch.float32, device=dev)
-    o_seq = torch.empty_like(q_seq)
-    ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
-    if w.backward:
-        do_all = torch.empty_like(q_all)
-        dq_all, dk_all, dv_all = torch.empty_like(q_all), torch.empty_like(k_all), torch.empty_like(v_all)
-        dq_seq, dk_seq, dv_seq = torch.empty_like(q_seq), torch.empty_like(k_seq), torch.empty_like(v_seq)
-
     stream = torch.cuda.current_stream(dev)
-    ev = {"attn_fwd": [], "attn_bwd": [], "relayout": []}
-    launches = {"n": 0}
-
-    def timed(kind, fn):
-        if args.kernel_events:
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            ev[kind].append((a, b))
-        else:
-            fn()
-
-    def step(record: bool):
-        # first all-to-all: every rank's head slice of Q, K, V
-        timed("relayout", lambda: U.seq_to_head(q_seq, P, out=q_all))
-        timed("relayout", lambda: U.seq_to_head(k_seq, P, out=k_all))
-        timed("relayout", lambda: U.seq_to_head(v_seq, P, out=v_all))
-        n = 3
-        for r in range(P):
-            timed("attn_fwd", lambda: U.attn_fwd(q_all[r], k_all[r], v_all[r], pos, out=o_all[r],
-                                                 lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws))
-            n += 4
-        if w.backward:
-            timed("relayout", lambda: U.seq_to_head(do_seq, P, out=do_all))
-            n += 1
-            for r in range(P):
-                timed("attn_bwd", lambda: U.attn_bwd(q_all[r], k_all[r], v_all[r], o_all[r], do_all[r],
-                                                     lse_all[r * Hl:(r + 1) * Hl], pos, ws=ws, dq=dq_all[r],
-                                                     dk=dk_all[r], dv=dv_all[r]))
-                n += BWD_LAUNCHES
-            timed("relayout", lambda: U.head_to_seq(dq_all, P, out=dq_seq))
-            timed("relayout", lambda: U.head_to_seq(dk_all, P, out=dk_seq))
-            timed("relayout", lambda: U.head_to_seq(dv_all, P, out=dv_seq))
-            n += 3
-        # second all-to-all: O back to sequence shards
-        timed("relayout", lambda: U.head_to_seq(o_all, P, out=o_seq))
-        n += 1
-        if record:
-            launches["n"] += n
+    timed = Timer(stream, False)
+    if world == 1:
+        step, launches_per_step, ws = build_single(U, w, inp, dev, timed)
+    else:
+        step, launches_per_step, ws = build_multi(U, w, inp, dev, timed, world, rank)
+        for key in ("q", "k", "v", "do"):
+            inp.pop(key, None)     # each rank keeps only its shard
+        torch.cuda.empty_cache()
 
     # warm-up
-    saved = args.kernel_events
-    args.kernel_events = False
     for _ in range(args.warmup):
-        step(False)
+        step()
     torch.cuda.synchronize()
-    U.sync_status(ws)
-    args.kernel_events = saved
+    U.sync_status(ws)        # raises if a bounded device wait ran out
+    timed.enabled = args.kernel_events
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -246,7 +302,7 @@ def run_gpu(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        step(True)
+        step()
     t1.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
@@ -260,26 +316,21 @@ def run_gpu(args):
         ms_total = float(t.item())
     ms_step = ms_total / args.steps
 
-    def avg_ms(kind):
-        xs = [a.elapsed_time(b) for a, b in ev[kind]]
-        return (sum(xs) / len(xs)) if xs else None, (sum(xs) if xs else None)
+    fwd_avg, _ = timed.stats("attn_fwd")
+    bwd_avg, _ = timed.stats("attn_bwd")
+    _, rel_sum = timed.stats("relayout")
+    _, exch_sum = timed.stats("exchange")
 
-    fwd_avg, fwd_sum = avg_ms("attn_fwd")
-    bwd_avg, bwd_sum = avg_ms("attn_bwd")
-    rel_avg, rel_sum = avg_ms("relayout")
-
-    total_flop = (fwd_flop + bwd_flop) * world
+    total_flop = fwd_flop + bwd_flop          # the whole job (all ranks, all heads)
     value = total_flop / (ms_step * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
     long_step = ms_total > 1000.0
     bf16_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
-    fwd_flop_launch = fwd_flop / P                     # one launch = one rank's heads
+    launches_attn_fwd = (w.P if world == 1 else 1) * world    # attention launches per step over the job
+    fwd_flop_launch = fwd_flop / launches_attn_fwd
     achieved = fwd_flop_launch / (fwd_avg * 1e-3) / 1e12 if fwd_avg else None
-    traffic = lookup_traffic("attn_fwd_kernel", w.name)
-
-    # ---- end to end through the public API with host buffers (rank 0 of P only
-    # would understate the copies; the whole job's inputs cross PCIe each step)
-    e2e = run_e2e(U, w, inp, args, dev) if args.e2e_steps > 0 else None
+    traffic = lookup_traffic("attn_fwd_kernel", w.name) if world == 1 else None
+    e2e = run_e2e(U, w, inp, args, dev) if (args.e2e_steps > 0 and world == 1) else None
 
     out = {
         "metric": METRIC,
@@ -290,17 +341,20 @@ def run_gpu(args):
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if world > 1 else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": w.name, "N": N, "P": P, "H": w.H, "Hkv": w.Hkv, "d": d, "docs": w.docs,
-            "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
-            "step": "seq_to_head(Q,K,V) for all P ranks; attn_fwd for each rank's head slice"
-                    + ("; seq_to_head(dO), attn_bwd per rank, head_to_seq(dQ,dK,dV)" if w.backward else "")
-                    + "; head_to_seq(O) for all ranks",
-            "l2": "inputs larger than L2 (126 MB): Q alone is %d MiB" % (N * w.H * d * 2 >> 20),
+            "workload": w.name, "N": w.N, "P": w.P if world == 1 else world, "H": w.H, "Hkv": w.Hkv, "d": w.d,
+            "docs": w.docs, "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
+            "step": (("seq_to_head(Q,K,V) for all P ranks; attn_fwd for each rank's head slice"
+                      + ("; seq_to_head(dO), attn_bwd per rank, head_to_seq(dQ,dK,dV)" if w.backward else "")
+                      + "; head_to_seq(O) for all ranks") if world == 1 else
+                     ("Ulysses over %d GPUs: pack + NCCL all-to-all of Q,K,V; attn_fwd on N x H/%d heads"
+                      % (world, world) + ("; dO exchange, attn_bwd, dQ/dK/dV exchanges" if w.backward else "")
+                      + "; O exchange + unpack")),
+            "l2": "inputs larger than L2 (126 MB): Q alone is %d MiB" % (w.N * w.H * w.d * 2 >> 20),
         },
         "roofline": {
             "kernel": "attn_fwd_kernel (timed with the doc-bounds scan it is launched with)",
@@ -314,24 +368,24 @@ def run_gpu(args):
             "traffic": traffic,
             "flop_per_launch": fwd_flop_launch,
         },
-        "relayout": {
-            "bytes_per_step": relayout_bytes,
-            "ms_per_step": round(rel_sum / args.steps, 4) if rel_sum else None,
-            "achieved_gbs": round(relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9, 1) if rel_sum else None,
-            "peak_gbs": peaks["hbm_gbs"],
-            "frac": round(relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if rel_sum else None,
-            "frac_of_spec_8000": round(relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9 / SPEC_HBM_GBS, 4) if rel_sum else None,
-        },
         "attn_fwd_ms_per_launch": round(fwd_avg, 4) if fwd_avg else None,
         "attn_bwd_ms_per_launch": round(bwd_avg, 4) if bwd_avg else None,
-        "attn_bwd_tflops": round((bwd_flop / P) / (bwd_avg * 1e-3) / 1e12, 2) if bwd_avg else None,
-        "gpu_launches": launches["n"],
+        "attn_bwd_tflops": round((bwd_flop / launches_attn_fwd) / (bwd_avg * 1e-3) / 1e12, 2) if bwd_avg else None,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
     }
+    if rel_sum:
+        rb = relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9
+        out["relayout"] = {"bytes_per_step": relayout_bytes, "ms_per_step": round(rel_sum / args.steps, 4),
+                           "achieved_gbs": round(rb, 1), "peak_gbs": peaks["hbm_gbs"],
+                           "frac": round(rb / peaks["hbm_gbs"], 4), "frac_of_spec_8000": round(rb / SPEC_HBM_GBS, 4)}
+    if exch_sum:
+        out["exchange_ms_per_step"] = round(exch_sum / args.steps, 4)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, inp, args)
     if dist is not None:
+        dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)

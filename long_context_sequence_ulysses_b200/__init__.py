@@ -6,7 +6,7 @@ dtypes, allocate outputs and workspace through torch (device memory and
 streams are torch's job), and call the C ABI on the current CUDA stream.
 Every step of the computation runs in the library's CUDA kernels; there is no
 fallback, and importing the package fails if the library has not been built
-(``python -m long_context_sequence_ulysses_b200.build``).
+(``python long_context_sequence_ulysses_b200/build.py``).
 
 The method (page "Hugging Face并行加速：10倍提升超长序列训练效率", section
 "Ulysses的工作原理"): N tokens are split over P ranks; an all-to-all gives each
@@ -25,7 +25,7 @@ import torch
 
 __all__ = [
     "UlyssesError", "library_path", "seq_to_head", "head_to_seq", "workspace_bytes", "attn_fwd",
-    "attn_fwd_fused", "attn_bwd", "sync_status", "set_wait_limit_ns", "version",
+    "attn_fwd_fused", "attn_bwd", "sync_status", "set_wait_limit_ns", "set_debug_flags", "version",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -48,7 +48,7 @@ class UlyssesError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
-            f"{_LIB_PATH} is missing: build it with `python -m long_context_sequence_ulysses_b200.build` "
+            f"{_LIB_PATH} is missing: build it with `python long_context_sequence_ulysses_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(_LIB_PATH)
     P, I64, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
@@ -64,6 +64,8 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_sync_status.argtypes = [P, P]
     lib.ulysses_set_wait_limit_ns.argtypes = [I64]
     lib.ulysses_set_wait_limit_ns.restype = None
+    lib.ulysses_set_debug_flags.argtypes = [ctypes.c_uint32]
+    lib.ulysses_set_debug_flags.restype = None
     for name in ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_fwd_fused",
                  "ulysses_attn_bwd", "ulysses_sync_status"):
         getattr(lib, name).restype = I32
@@ -238,6 +240,11 @@ def sync_status(ws: torch.Tensor) -> None:
 
 def set_wait_limit_ns(ns: int) -> None:
     _lib.ulysses_set_wait_limit_ns(int(ns))
+
+
+def set_debug_flags(flags: int) -> None:
+    """Test hook: bit 0 makes later forward launches run one bounded wait out."""
+    _lib.ulysses_set_debug_flags(int(flags))
 
 
 def default_scale(d: int) -> float:

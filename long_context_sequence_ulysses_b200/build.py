@@ -1,6 +1,8 @@
 """Build libulysses.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m long_context_sequence_ulysses_b200.build [--force] [--verbose]
+    python long_context_sequence_ulysses_b200/build.py [--force] [--verbose] [--ptxas-info]
+
+(Run it by path: importing the package loads the library it builds.)
 
 Each .cu file under csrc/ is compiled to an object in _build/ (in parallel),
 then linked into long_context_sequence_ulysses_b200/libulysses.so. Objects are

@@ -19,6 +19,7 @@ namespace {
 
 thread_local char g_err[512] = "";
 int64_t g_wait_limit_ns = 1000000000LL;
+uint32_t g_debug_flags = 0;
 
 int fail(int code, const char *fmt, ...)
 {
@@ -107,6 +108,8 @@ const char *ulysses_version(void) { return "ulysses-b200 0.1 (sm_100a)"; }
 
 void ulysses_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns = ns > 0 ? ns : 1000000000LL; }
 
+void ulysses_set_debug_flags(uint32_t flags) { g_debug_flags = flags; }
+
 static int relayout_common(bool to_head, const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
                            void *stream)
 {
@@ -192,6 +195,7 @@ static int attn_fwd_common(const char *name, const void *q, const void *k, const
     a.ws = static_cast<const char *>(ws);
     a.L = L;
     a.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
+    a.debug_flags = g_debug_flags;
     e = launch_attn_fwd(a, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return ULYSSES_OK;

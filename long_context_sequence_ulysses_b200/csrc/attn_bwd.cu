@@ -12,7 +12,7 @@
 // 10倍提升超长序列训练效率", section "Ulysses的工作原理").
 //
 // Three kernels, all deterministic (no atomics):
-//  1. prep: D_i and LSE_i*log2(e) per (head, row) into a 128-padded layout.
+//  1. prep: D_i and -LSE_i*log2(e) per (head, row) into a 128-padded layout.
 //  2. dK/dV: one CTA per (key tile, KV head) loops over the query heads of the
 //     GQA group and the query tiles that see the key tile:
 //       S^T = K Q^T, dP^T = V dO^T       (SS MMA, M = keys, N = queries)
@@ -43,7 +43,7 @@ struct BwdParams {
     const int32_t *kv_qend;
     const int32_t *kv_order;
     const float *delta;   // [Hl][Npad]
-    const float *lse2;    // [Hl][Npad]
+    const float *lse2;    // [Hl][Npad]: -LSE * log2(e) (-inf on padding rows)
     __nv_bfloat16 *dq, *dk, *dv;
     int N, Npad, T, Hl, Hkvl;
     float scale_log2, scale;
@@ -96,7 +96,7 @@ __device__ __forceinline__ float dot8_bf16(const uint4 &a, const uint4 &b)
     return acc;
 }
 
-// D_i = sum_c dO_ic O_ic and LSE_i * log2(e), one warp per (head, padded row).
+// D_i = sum_c dO_ic O_ic and -LSE_i * log2(e), one warp per (head, padded row).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
                                                       const __nv_bfloat16 *__restrict__ dout,
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
         delta[w] = i < N ? acc : 0.f;
-        lse2[w] = i < N ? lse[static_cast<int64_t>(h) * N + i] * kLog2e : CUDART_INF_F;
+        lse2[w] = i < N ? -lse[static_cast<int64_t>(h) * N + i] * kLog2e : -CUDART_INF_F;
     }
 }
 
@@ -242,36 +242,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        {   // the whole warp runs the loop; elect.sync picks the issuing lane
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
-            bool ok = mbar_wait(kv_full, 0, wc);
+            bool ok = mbar_wait_warp(kv_full, 0, wc);
             for (int it = 0; ok && it < n_it; ++it) {
                 const int s = it % C::NST, u = it / C::NST;
-                if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
+                if (!mbar_wait_warp(&qdo_full[s], u & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tbase + C::T_S, kmajor_desc<D>(aK, kk), kmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
+                    umma_ss_elect(tbase + C::T_S, kmajor_desc<D>(aK, kk), kmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
                             C::IDESC_SS, kk > 0 ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tbase + C::T_DP, kmajor_desc<D>(aV, kk), kmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
+                    umma_ss_elect(tbase + C::T_DP, kmajor_desc<D>(aV, kk), kmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
                             C::IDESC_SS, kk > 0 ? 1u : 0u);
-                umma_commit(s_full);
-                if (!mbar_wait(ds_full, it & 1, wc)) { ok = false; break; }
+                umma_commit_elect(s_full);
+                if (!mbar_wait_warp(ds_full, it & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTileM / 16; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
+                    umma_ts_elect(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
                             C::IDESC_TS, acc);   // dV += P^T dO
-                    umma_ts(tbase + C::T_ACC1, tbase + C::T_DP + kk * 8, mnmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
+                    umma_ts_elect(tbase + C::T_ACC1, tbase + C::T_DP + kk * 8, mnmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
                             C::IDESC_TS, acc);   // dK += dS^T Q
                 }
-                umma_commit(&qdo_empty[s]);
+                umma_commit_elect(&qdo_empty[s]);
             }
-            if (ok) umma_commit(acc_done);
-            umma_commit(mma_done);
+            if (ok) umma_commit_elect(acc_done);
+            umma_commit_elect(mma_done);
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(mma_done, 0, drain);
         }
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!mbar_wait(s_full, it & 1, wc)) { ok = false; break; }
             if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const float *rl = sRow + (s * 2 + 0) * 128;
-            const float *rd = sRow + (s * 2 + 1) * 128;
+            const float *rl = sRow + (s * 2 + 0) * 128;   // -lse2 of the 128 queries
+            const float *rd = sRow + (s * 2 + 1) * 128;   // delta of the 128 queries
             const bool need_mask = (q0 < j) || (q0 + kTileM - 1 >= dend);
             const bool any_mask = __any_sync(0xffffffffu, need_mask);
 #pragma unroll
@@ -310,21 +310,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld_wait();
                 uint32_t pp[32], dd[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float pv[2], dv[2];
+                for (int e = 0; e < 32; e += 2) {
+                    const int c = half * 64 + 2 * e;   // columns c .. c+3
+                    const float4 nl = *reinterpret_cast<const float4 *>(rl + c);
+                    const float4 dl = *reinterpret_cast<const float4 *>(rd + c);
+                    float x[4], pv[4], t[4], dv[4];
+                    fma2(x[0], x[1], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, nl.x, nl.y);
+                    fma2(x[2], x[3], __uint_as_float(sr[2 * e + 2]), __uint_as_float(sr[2 * e + 3]), sl2, sl2, nl.z,
+                         nl.w);
+                    if (any_mask) {
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int c = half * 64 + 2 * e + k;
-                        float x = __uint_as_float(sr[2 * e + k]);
-                        if (any_mask) {
-                            const int qi = q0 + c;
-                            if (qi < j || qi >= dend) x = -CUDART_INF_F;
+                        for (int k = 0; k < 4; ++k) {
+                            const int qi = q0 + c + k;
+                            if (qi < j || qi >= dend) x[k] = -CUDART_INF_F;
                         }
-                        pv[k] = ex2_approx(fmaf(x, sl2, -rl[c]));
-                        dv[k] = pv[k] * (__uint_as_float(dr[2 * e + k]) - rd[c]);
                     }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) pv[k] = ex2_approx(x[k]);
+                    sub2(t[0], t[1], __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), dl.x, dl.y);
+                    sub2(t[2], t[3], __uint_as_float(dr[2 * e + 2]), __uint_as_float(dr[2 * e + 3]), dl.z, dl.w);
+                    mul2(dv[0], dv[1], pv[0], pv[1], t[0], t[1]);
+                    mul2(dv[2], dv[3], pv[2], pv[3], t[2], t[3]);
                     pp[e] = pack_bf16x2(pv[0], pv[1]);
+                    pp[e + 1] = pack_bf16x2(pv[2], pv[3]);
                     dd[e] = pack_bf16x2(dv[0], dv[1]);
+                    dd[e + 1] = pack_bf16x2(dv[2], dv[3]);
                 }
                 tmem_st32(tbase + C::T_S + lane_off + half * 32, pp);    // P^T  (queries packed in pairs)
                 tmem_st32(tbase + C::T_DP + lane_off + half * 32, dd);   // dS^T
@@ -443,32 +453,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (last_use[s] >= 0) mbar_wait(&kv_full[s], last_use[s] & 1, drain);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {   // the whole warp runs the loop; elect.sync picks the issuing lane
             const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
-            bool ok = mbar_wait(qdo_full, 0, wc);
+            bool ok = mbar_wait_warp(qdo_full, 0, wc);
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int s = j % C::NST, u = j / C::NST;
-                if (!mbar_wait(&kv_full[s], u & 1, wc)) { ok = false; break; }
+                if (!mbar_wait_warp(&kv_full[s], u & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tbase + C::T_S, kmajor_desc<D>(aQ, kk), kmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
+                    umma_ss_elect(tbase + C::T_S, kmajor_desc<D>(aQ, kk), kmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
                             C::IDESC_SS, kk > 0 ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tbase + C::T_DP, kmajor_desc<D>(aDO, kk), kmajor_desc<D>(aV + s * C::TILE_BYTES, kk),
+                    umma_ss_elect(tbase + C::T_DP, kmajor_desc<D>(aDO, kk), kmajor_desc<D>(aV + s * C::TILE_BYTES, kk),
                             C::IDESC_SS, kk > 0 ? 1u : 0u);
-                umma_commit(s_full);
-                if (!mbar_wait(ds_full, j & 1, wc)) { ok = false; break; }
+                umma_commit_elect(s_full);
+                if (!mbar_wait_warp(ds_full, j & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTileN / 16; ++kk)
-                    umma_ts(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
+                    umma_ts_elect(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
                             C::IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);   // dQ += dS K
-                umma_commit(&kv_empty[s]);
+                umma_commit_elect(&kv_empty[s]);
             }
-            if (ok) umma_commit(acc_done);
-            umma_commit(mma_done);
+            if (ok) umma_commit_elect(acc_done);
+            umma_commit_elect(mma_done);
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(mma_done, 0, drain);
         }
@@ -478,7 +488,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int i = qt * kTileM + r;
         const bool valid = i < p.N;
         const int lo = valid ? p.doc_start[i] : i;
-        const float l2 = p.lse2[static_cast<int64_t>(h) * p.Npad + i];
+        const float nl2 = p.lse2[static_cast<int64_t>(h) * p.Npad + i];   // -LSE * log2(e)
         const float di = p.delta[static_cast<int64_t>(h) * p.Npad + i];
         const float sl2 = p.scale_log2;
         bool ok = true;
@@ -497,19 +507,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 uint32_t dd[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    float dv[2];
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int c = half * 64 + 2 * e + k;
-                        float x = __uint_as_float(sr[2 * e + k]);
-                        if (any_mask) {
-                            const int key = c0 + c;
-                            if (key < lo || key > i) x = -CUDART_INF_F;
-                        }
-                        const float pv = ex2_approx(fmaf(x, sl2, -l2));
-                        dv[k] = pv * (__uint_as_float(dr[2 * e + k]) - di);
+                    const int c = half * 64 + 2 * e;
+                    float x0, x1;
+                    fma2_bcast(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, nl2);
+                    if (any_mask) {
+                        if (c0 + c < lo || c0 + c > i) x0 = -CUDART_INF_F;
+                        if (c0 + c + 1 < lo || c0 + c + 1 > i) x1 = -CUDART_INF_F;
                     }
-                    dd[e] = pack_bf16x2(dv[0], dv[1]);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    float t0, t1, d0, d1;
+                    sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), di, di);
+                    mul2(d0, d1, p0, p1, t0, t1);
+                    dd[e] = pack_bf16x2(d0, d1);
                 }
                 tmem_st32(tbase + C::T_S + lane_off + half * 32, dd);   // dS (keys packed in pairs)
             }

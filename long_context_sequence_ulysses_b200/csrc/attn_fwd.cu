@@ -62,6 +62,7 @@ struct FwdParams {
     float scale_log2;      // softmax scale * log2(e)
     uint32_t *status;
     uint64_t wait_limit_ns;
+    uint32_t debug_flags;   // bit 0: CTA 0 waits on a barrier nobody arrives on (tests the timeout path)
 };
 
 template <int D>
@@ -77,7 +78,7 @@ struct FwdCfg {
     static constexpr int OFF_K = 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + NST * TILE_BYTES;
-    static constexpr int NBAR = 2 + 4 * NST + 2 + 2 + 2 + 1;
+    static constexpr int NBAR = 2 + 4 * NST + 2 + 2 + 2 + 1 + 1;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kTileM, kTileN, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kTileM, D, false, true);
@@ -107,7 +108,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t *p_full = s_full + 2;           // [2] per tile
     uint64_t *o_done = p_full + 2;           // [2] per tile
     uint64_t *mma_done = o_done + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *never = mma_done + 1;          // never arrived on (timeout test only)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(never + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -141,6 +143,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(&o_done[x], 1);
         }
         mbar_init(mma_done, 1);
+        mbar_init(never, 1);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
@@ -289,6 +292,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float ms = -CUDART_INF_F;   // exponent offset in use (scaled log2 units)
         float l = 0.f;
         bool ok = true;
+        if ((p.debug_flags & 1u) && blockIdx.x == 0 && x == 0) ok = mbar_wait(never, 0, wc);   // runs out
         for (int it = 0; it < n_it; ++it) {
             if (!mbar_wait(&s_full[x], it & 1, wc)) { ok = false; break; }
             tc_fence_after();
@@ -424,6 +428,7 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.status = reinterpret_cast<uint32_t *>(const_cast<char *>(a.ws) + a.L.status);
     p.wait_limit_ns = a.wait_limit_ns;
+    p.debug_flags = a.debug_flags;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);

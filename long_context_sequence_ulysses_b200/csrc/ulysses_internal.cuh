@@ -82,6 +82,7 @@ struct FwdLaunch {
     const char *ws;
     WsLayout L;
     uint64_t wait_limit_ns;
+    uint32_t debug_flags;
 };
 cudaError_t launch_attn_fwd(const FwdLaunch &a, cudaStream_t stream);
 

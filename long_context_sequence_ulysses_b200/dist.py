@@ -30,46 +30,60 @@ def _world(group) -> Tuple[int, int]:
     return dist.get_world_size(group), dist.get_rank(group)
 
 
-def _cuda_pack(x: torch.Tensor, G: int) -> torch.Tensor:
+def _cuda_pack(x: torch.Tensor, G: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     import long_context_sequence_ulysses_b200 as U
-    return U.seq_to_head(x, G)
+    return U.seq_to_head(x, G, out=out)
 
 
-def _cuda_unpack(y: torch.Tensor, G: int) -> torch.Tensor:
+def _cuda_unpack(y: torch.Tensor, G: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     import long_context_sequence_ulysses_b200 as U
-    return U.head_to_seq(y, G)
+    return U.head_to_seq(y, G, out=out)
 
 
 def seq_to_head(x_local: torch.Tensor, group=None,
-                pack: Optional[Callable[[torch.Tensor, int], torch.Tensor]] = None) -> torch.Tensor:
-    """[N/G][Hx][d] sequence shard -> [N][Hx/G][d] head slice of this rank."""
+                pack: Optional[Callable] = None, send: Optional[torch.Tensor] = None,
+                recv: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """[N/G][Hx][d] sequence shard -> [N][Hx/G][d] head slice of this rank.
+    ``send`` / ``recv`` are optional preallocated [G][N/G][Hx/G][d] buffers."""
     G, _ = _world(group)
     n_loc, Hx, d = x_local.shape
     if Hx % G or n_loc % G:
         raise ValueError(f"heads ({Hx}) and local tokens ({n_loc}) must be divisible by the group size {G}")
-    send = (pack or _cuda_pack)(x_local, G)                     # [G][N/G][Hx/G][d]
-    recv = torch.empty_like(send)
+    if pack is None:
+        send = _cuda_pack(x_local, G, out=send)                  # [G][N/G][Hx/G][d]
+    else:
+        send = pack(x_local, G)
+    if recv is None:
+        recv = torch.empty_like(send)
     dist.all_to_all_single(recv.view(torch.uint8), send.contiguous().view(torch.uint8), group=group)
     return recv.view(G * n_loc, Hx // G, d)
 
 
 def head_to_seq(y: torch.Tensor, group=None,
-                unpack: Optional[Callable[[torch.Tensor, int], torch.Tensor]] = None) -> torch.Tensor:
-    """[N][Hx/G][d] head slice -> [N/G][Hx][d] sequence shard of this rank."""
+                unpack: Optional[Callable] = None, recv: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """[N][Hx/G][d] head slice -> [N/G][Hx][d] sequence shard of this rank.
+    ``recv`` ([G][N/G][Hx/G][d]) and ``out`` ([N/G][Hx][d]) may be preallocated."""
     G, _ = _world(group)
     N, Hl, d = y.shape
     if N % G:
         raise ValueError(f"N ({N}) must be divisible by the group size {G}")
     send = y.contiguous().view(G, N // G, Hl, d)                # block r goes to rank r
-    recv = torch.empty_like(send)
+    if recv is None:
+        recv = torch.empty_like(send)
     dist.all_to_all_single(recv.view(torch.uint8), send.view(torch.uint8), group=group)
-    return (unpack or _cuda_unpack)(recv, G)                     # [N/G][Hx][d]
+    if unpack is None:
+        return _cuda_unpack(recv, G, out=out)                    # [N/G][Hx][d]
+    return unpack(recv, G)
 
 
-def gather_position_ids(pos_local: torch.Tensor, group=None) -> torch.Tensor:
+def gather_position_ids(pos_local: torch.Tensor, group=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """All ranks' position ids, in sequence order (each rank needs the whole
     sequence's document structure once it holds whole-sequence head slices)."""
     G, _ = _world(group)
+    if out is not None and pos_local.is_cuda:
+        dist.all_gather_into_tensor(out, pos_local.contiguous(), group=group)
+        return out
     parts = [torch.empty_like(pos_local) for _ in range(G)]
     dist.all_gather(parts, pos_local.contiguous(), group=group)
     return torch.cat(parts)
