@@ -24,7 +24,9 @@
 // The softmax reads its S row, masks only diagonal / document-boundary tiles,
 // keeps a running max with lazy rescaling (O and l are rescaled only when the
 // max grows by more than 2^8), and writes P = exp2(...) back as bf16. The
-// row arithmetic uses the packed fp32x2 FMA / add and the 3-input max.
+// row arithmetic uses the packed fp32x2 FMA / add and the 3-input max; 3/8
+// of the exponentials are evaluated on the FMA pipe (ex2_poly2) so that the
+// special-function unit is not the limit.
 // Key tiles outside [doc_start(first row), last row] of a tile are never
 // visited by that tile.
 #include "ptx.cuh"
@@ -41,6 +43,11 @@ constexpr int kFwdThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
+// Column pairs (out of every 8) whose exponentials run on the FMA pipe: the
+// SFU needs 8 cycles per warp instruction, so with only SFU exponentials a
+// 128-column row costs 1024 SFU cycles per warp against ~400 issue slots of
+// other work; moving 3/8 of them to packed polynomials balances the two.
+constexpr int kEmuPairs = 3;
 // Register split: launched at 168 per thread (384 x 168 = 64512); the two
 // softmax warpgroups take 224, the producer / MMA warpgroup keeps 56:
 // 256 x 224 + 128 x 56 = 64512.
@@ -355,8 +362,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 64; ++e) {
                 float x0, x1;
                 fma2_bcast(x0, x1, s[2 * e], s[2 * e + 1], sl2, -moff);
-                const float e0 = ex2_approx(x0);
-                const float e1 = ex2_approx(x1);
+                // 3 column pairs in 8 take the FMA-pipe exponential, the rest the SFU
+                float e0, e1;
+                if ((e & 7) < kEmuPairs) {
+                    ex2_poly2(e0, e1, x0, x1);
+                } else {
+                    e0 = ex2_approx(x0);
+                    e1 = ex2_approx(x1);
+                }
                 add2_acc(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], e0, e1);
                 pk[e] = pack_bf16x2(e0, e1);
             }

@@ -367,6 +367,39 @@ __device__ __forceinline__ float ex2_poly(float x)
     return __int_as_float(__float_as_int(p) + (j << 23));
 }
 
+// Two exponentials at once with ex2_poly's method, on packed fp32x2 FMAs.
+// 2^j is inserted with one integer multiply-add: t = x + 1.5*2^23 holds
+// round(x) in its low mantissa bits, and bits(t) << 23 == round(x) << 23
+// (mod 2^32) because 0x4B400000 << 23 wraps to 0.
+__device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0, float x1)
+{
+    x0 = fmaxf(x0, -125.0f);
+    x1 = fmaxf(x1, -125.0f);
+    float t0, t1, r0, r1, f0, f1, p0, p1;
+    asm("{\n\t.reg .b64 rx, rm, rt, rr, rf, rp, c3, c2, c1, c0;\n\t"
+        "mov.b64 rx, {%8, %9};\n\t"
+        "mov.b64 rm, {%10, %10};\n\t"
+        "add.rn.f32x2 rt, rx, rm;\n\t"
+        "sub.rn.f32x2 rr, rt, rm;\n\t"
+        "sub.rn.f32x2 rf, rx, rr;\n\t"
+        "mov.b64 c3, {%11, %11};\n\t"
+        "mov.b64 c2, {%12, %12};\n\t"
+        "mov.b64 c1, {%13, %13};\n\t"
+        "mov.b64 c0, {%14, %14};\n\t"
+        "fma.rn.f32x2 rp, c3, rf, c2;\n\t"
+        "fma.rn.f32x2 rp, rp, rf, c1;\n\t"
+        "fma.rn.f32x2 rp, rp, rf, c0;\n\t"
+        "mov.b64 {%0, %1}, rt;\n\t"
+        "mov.b64 {%2, %3}, rr;\n\t"
+        "mov.b64 {%4, %5}, rf;\n\t"
+        "mov.b64 {%6, %7}, rp;\n\t}"
+        : "=f"(t0), "=f"(t1), "=f"(r0), "=f"(r1), "=f"(f0), "=f"(f1), "=f"(p0), "=f"(p1)
+        : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(0.0551716685295105f), "f"(0.2426111251115799f),
+          "f"(0.6932609677314758f), "f"(0.9999280571937561f));
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Packed fp32 pair arithmetic (two lanes per instruction, IEEE round to
 // nearest): (d0, d1) = (a0, a1) * b + c with b and c broadcast.
 __device__ __forceinline__ void fma2_bcast(float &d0, float &d1, float a0, float a1, float b, float c)

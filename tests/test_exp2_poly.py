@@ -24,8 +24,28 @@ def _device_coefficients():
     return np.array([c0, c1, c2, c3], dtype=np.float32)
 
 
+def _packed_device_coefficients():
+    src = open(PTX).read()
+    body = src[src.index("void ex2_poly2("):]
+    body = body[:body.index("y0 = ")]
+    lits = [float(v) for v in re.findall(r"([0-9]\.[0-9]+)f", body)]
+    c3, c2, c1, c0 = lits[-4:]                      # operand order: c3, c2, c1, c0
+    return np.array([c0, c1, c2, c3], dtype=np.float32)
+
+
 def test_coefficients_match_the_fit():
     assert np.array_equal(_device_coefficients(), exp2_poly.fp32_coefficients())
+    assert np.array_equal(_packed_device_coefficients(), exp2_poly.fp32_coefficients())
+
+
+def test_packed_exponent_insertion_is_the_same():
+    # the packed form adds bits(t) << 23 instead of (bits(t) - 0x4B400000) << 23
+    x = np.linspace(-125, 8, 200001, dtype=np.float32)
+    t = (x + np.float32(12582912.0)).astype(np.float32)
+    tb = t.view(np.int32).astype(np.int64)
+    a = (tb << 23) & 0xFFFFFFFF
+    b = ((tb - 0x4B400000) << 23) & 0xFFFFFFFF
+    assert np.array_equal(a, b)
 
 
 def test_relative_error_bound():
