@@ -39,7 +39,7 @@ extern "C" {
 typedef enum {
     ULYSSES_OK = 0,
     ULYSSES_ERR_INVALID = -1,     /* null or misaligned pointer, H % P, Hkv % P, N % P, H % Hkv, d, ... */
-    ULYSSES_ERR_UNSUPPORTED = -2, /* a valid request this build does not implement */
+    ULYSSES_ERR_UNSUPPORTED = -2, /* a valid request the library does not implement */
     ULYSSES_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
     ULYSSES_ERR_TIMEOUT = -4,     /* a bounded device-side wait ran out */
     ULYSSES_ERR_WORKSPACE = -5    /* workspace missing or smaller than ulysses_attn_workspace_bytes() */
