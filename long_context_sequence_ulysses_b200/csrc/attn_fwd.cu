@@ -11,8 +11,10 @@
 // one head; they share every K/V tile load.
 //   warps 0..3   softmax warpgroup of tile A (thread t owns row t = TMEM lane t)
 //   warps 4..7   softmax warpgroup of tile B
-//   warp 8       TMA producer: Q_A, Q_B, then K and V tiles into an NST-stage ring
-//   warp 9       allocates tensor memory; lane 0 issues every tcgen05.mma
+//   warp 8       TMA producer: Q_A, Q_B, then the K tiles into a KST-stage ring
+//   warp 9       allocates tensor memory; issues every tcgen05.mma (one elected lane)
+//   warp 10      TMA producer of the V tiles (VST-stage ring; a V tile is held one
+//                step longer than its K tile, so it gets the extra stage)
 // Tensor memory (512 columns): S_A at 0, S_B at 128 (fp32 128x128 each; the
 // bf16 probabilities P overwrite the first 64 columns of their own S), O_A at
 // 256, O_B at 256 + d.
@@ -42,6 +44,7 @@ namespace {
 constexpr int kFwdThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;
 constexpr uint32_t kTmemCols = 512;
 // Column pairs (out of every 8) whose exponentials run on the FMA pipe: the
 // SFU needs 8 cycles per warp instruction, so with only SFU exponentials a
@@ -79,13 +82,14 @@ struct FwdCfg {
     static constexpr int NA = D / AW;                         // atoms along d
     static constexpr int ATOM_BYTES = kTileM * SW;            // one 128-row atom block
     static constexpr int TILE_BYTES = kTileM * D * 2;         // a Q, K or V tile
-    static constexpr int NST = (D == 128) ? 2 : 4;            // K/V pipeline stages
+    static constexpr int KST = (D == 128) ? 2 : 4;            // K pipeline stages
+    static constexpr int VST = (D == 128) ? 3 : 4;            // V pipeline stages
     static constexpr uint32_t SWZ = (SW == 128) ? kSwizzle128 : kSwizzle64;
     static constexpr int OFF_Q = 0;                           // Q_A, Q_B
     static constexpr int OFF_K = 2 * TILE_BYTES;
-    static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NST * TILE_BYTES;
-    static constexpr int NBAR = 2 + 4 * NST + 2 + 2 + 2 + 1 + 1;
+    static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
+    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 1;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;   // + alignment slack
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kTileM, kTileN, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kTileM, D, false, true);
@@ -107,11 +111,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint8_t *sV = smem + C::OFF_V;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars;                 // [2]
-    uint64_t *k_full = bars + 2;             // [NST]
-    uint64_t *k_empty = k_full + C::NST;
-    uint64_t *v_full = k_empty + C::NST;
-    uint64_t *v_empty = v_full + C::NST;
-    uint64_t *s_full = v_empty + C::NST;     // [2] per tile
+    uint64_t *k_full = bars + 2;             // [KST]
+    uint64_t *k_empty = k_full + C::KST;
+    uint64_t *v_full = k_empty + C::KST;     // [VST]
+    uint64_t *v_empty = v_full + C::VST;
+    uint64_t *s_full = v_empty + C::VST;     // [2] per tile
     uint64_t *p_full = s_full + 2;           // [2] per tile
     uint64_t *o_done = p_full + 2;           // [2] per tile
     uint64_t *mma_done = o_done + 2;
@@ -138,9 +142,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(&q_full[0], 1);
         mbar_init(&q_full[1], 1);
-        for (int s = 0; s < C::NST; ++s) {
+        for (int s = 0; s < C::KST; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::VST; ++s) {
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
@@ -172,7 +178,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
             for (int x = 0; x < (hasB ? 2 : 1); ++x) {
                 mbar_arrive_expect_tx(&q_full[x], C::TILE_BYTES);
 #pragma unroll
@@ -180,35 +185,46 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     tma_load_3d(sQ + x * C::TILE_BYTES + a * C::ATOM_BYTES, &tmQ, &q_full[x], a * C::AW,
                                 p.q_head0 + h, (x == 0 ? tA : tB) * kTileM);
             }
-            int last_k_use[C::NST], last_v_use[C::NST];
+            int last_use[C::KST];
 #pragma unroll
-            for (int s = 0; s < C::NST; ++s) last_k_use[s] = last_v_use[s] = -1;
+            for (int s = 0; s < C::KST; ++s) last_use[s] = -1;
             for (int j = 0; j < n_union; ++j) {
-                const int s = j % C::NST, u = j / C::NST;
-                const int key0 = (j0 + j) * kTileN;
+                const int s = j % C::KST, u = j / C::KST;
                 if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) break;
                 mbar_arrive_expect_tx(&k_full[s], C::TILE_BYTES);
 #pragma unroll
                 for (int a = 0; a < C::NA; ++a)
                     tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmK, &k_full[s], a * C::AW,
-                                p.kv_head0 + kvh, key0);
-                last_k_use[s] = u;
-                if (u > 0 && !mbar_wait(&v_empty[s], (u - 1) & 1, wc)) break;
-                mbar_arrive_expect_tx(&v_full[s], C::TILE_BYTES);
-#pragma unroll
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmV, &v_full[s], a * C::AW,
-                                p.kv_head0 + kvh, key0);
-                last_v_use[s] = u;
+                                p.kv_head0 + kvh, (j0 + j) * kTileN);
+                last_use[s] = u;
             }
             // Never leave the CTA with bulk copies still landing in its shared memory.
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(&q_full[0], 0, drain);
             if (hasB) mbar_wait(&q_full[1], 0, drain);
-            for (int s = 0; s < C::NST; ++s) {
-                if (last_k_use[s] >= 0) mbar_wait(&k_full[s], last_k_use[s] & 1, drain);
-                if (last_v_use[s] >= 0) mbar_wait(&v_full[s], last_v_use[s] & 1, drain);
+            for (int s = 0; s < C::KST; ++s)
+                if (last_use[s] >= 0) mbar_wait(&k_full[s], last_use[s] & 1, drain);
+        }
+    } else if (warp == kVProducerWarp) {
+        // ================================================================ V producer
+        if (lane == 0) {
+            prefetch_tmap(&tmV);
+            int last_use[C::VST];
+#pragma unroll
+            for (int s = 0; s < C::VST; ++s) last_use[s] = -1;
+            for (int j = 0; j < n_union; ++j) {
+                const int s = j % C::VST, u = j / C::VST;
+                if (u > 0 && !mbar_wait(&v_empty[s], (u - 1) & 1, wc)) break;
+                mbar_arrive_expect_tx(&v_full[s], C::TILE_BYTES);
+#pragma unroll
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmV, &v_full[s], a * C::AW,
+                                p.kv_head0 + kvh, (j0 + j) * kTileN);
+                last_use[s] = u;
             }
+            WaitCtx drain{p.wait_limit_ns, p.status, false};
+            for (int s = 0; s < C::VST; ++s)
+                if (last_use[s] >= 0) mbar_wait(&v_full[s], last_use[s] & 1, drain);
         }
     } else if (warp == kMmaWarp) {
         // ================================================================ MMA issuer
@@ -241,8 +257,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             bool ok = mbar_wait_warp(&q_full[0], 0, wc);
             if (ok && hasB) ok = mbar_wait_warp(&q_full[1], 0, wc);
             for (int j = 0; ok && j <= n_union; ++j) {
-                const int s = j % C::NST, u = j / C::NST;
-                const int sp = (j - 1 + C::NST) % C::NST, up = (j - 1) / C::NST;   // stage of key tile j-1
+                const int s = j % C::KST, u = j / C::KST;                            // K stage of key tile j
+                const int sp = (j - 1 + C::VST) % C::VST, up = (j - 1) / C::VST;   // V stage of key tile j-1
                 const bool have_j = j < n_union;
                 const bool pvA = (j - 1 >= 0) && (j - 1 < nA);
                 const bool sA = have_j && j < nA;
@@ -316,12 +332,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
             }
             const int c0 = (j0 + first_union + it) * kTileN;
-            const bool need_mask = (c0 < lo) || (c0 + kTileN - 1 > hi);
-            if (__any_sync(0xffffffffu, need_mask)) {
+            // This row may see key columns [cl, ch) of the tile. A row that sees
+            // none (its document starts in a later key tile: a tile straddling
+            // a document boundary) is zeroed through its exponent offset below;
+            // only rows cut inside the tile need a per-column mask.
+            const int cl = lo - c0, ch = hi - c0 + 1;
+            const bool row_out = cl >= kTileN;
+            if (__any_sync(0xffffffffu, !row_out && (cl > 0 || ch < kTileN))) {
+                // 32-column chunks valid for the whole warp are skipped; the
+                // others select column by column, branch-free.
 #pragma unroll
-                for (int c = 0; c < kTileN; ++c) {
-                    const int key = c0 + c;
-                    if (key < lo || key > hi) s[c] = -CUDART_INF_F;
+                for (int k = 0; k < kTileN / 32; ++k) {
+                    if (!__all_sync(0xffffffffu, cl <= 32 * k && ch >= 32 * k + 32)) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int c = 32 * k + e;
+                            s[c] = (c >= cl && c < ch) ? s[c] : -CUDART_INF_F;
+                        }
+                    }
                 }
             }
             // row max: 4 independent chains of 3-input max
@@ -330,7 +358,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int c = 4; c < kTileN; c += 8)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[c + e], s[c + 4 + e]);
-            const float mt = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+            const float mt = row_out ? -CUDART_INF_F : max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
             const float mt_s = mt * sl2;
             const bool resc = mt_s > ms + 8.0f;
             float alpha = 1.f;
@@ -352,7 +380,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     tmem_st32(tO + c * 32, raw);
                 }
             }
-            const float moff = (ms == -CUDART_INF_F) ? 0.f : ms;
+            // offset +inf turns every exponent of an all-masked row into exp2(-inf)
+            const float moff = row_out ? CUDART_INF_F : ((ms == -CUDART_INF_F) ? 0.f : ms);
             // P = exp2(s * scale*log2(e) - offset): the argument two columns at a
             // time (packed FMA), the exponential on the SFU, the row sum two
             // columns at a time (packed add, 4 independent accumulator pairs).
