@@ -7,11 +7,14 @@
 // communication, because heads are independent. Work stays O(n^2) but memory is
 // O(n) by tiling with an online softmax (section "超长序列训练的挑战").
 //
-// One CTA computes two consecutive 128-row query tiles A = 2u and B = 2u+1 of
-// one head; they share every K/V tile load.
+// The kernel is persistent: one CTA per SM takes work items from a global
+// counter, heaviest first. An item is two consecutive 128-row query tiles
+// A = 2u and B = 2u+1 of one head; they share every K/V tile load.
 //   warps 0..3   softmax warpgroup of tile A (thread t owns row t = TMEM lane t)
 //   warps 4..7   softmax warpgroup of tile B
-//   warp 8       TMA producer: Q_A, Q_B, then the K tiles into a KST-stage ring
+//   warp 8       takes the items and hands them to the other roles through a
+//                two-slot ring in shared memory; TMA producer of Q_A, Q_B and
+//                of the K tiles (KST-stage ring)
 //   warp 9       allocates tensor memory; issues every tcgen05.mma (one elected lane)
 //   warp 10      TMA producer of the V tiles (VST-stage ring; a V tile is held one
 //                step longer than its K tile, so it gets the extra stage)
@@ -21,6 +24,10 @@
 // The issue order ping-pongs the two tiles so that one warpgroup's softmax runs
 // while the tensor core works on the other tile:
 //     ... PV_A(j-1), S_A(j), PV_B(j-1), S_B(j), PV_A(j), S_A(j+1) ...
+// and runs on into the next item without a break: the K/V rings, the barrier
+// phases and the tensor memory carry over, the next item's Q tiles load as
+// soon as the last S of the current item has read them, and its first S
+// overlaps the current item's epilogue.
 // S = Q K^T is an SS MMA (both operands K-major in 128B-swizzled shared memory);
 // O += P V is a TS MMA (P from tensor memory, V MN-major from its TMA tile).
 // The softmax reads its S row, masks only diagonal / document-boundary tiles,
@@ -70,10 +77,40 @@ struct FwdParams {
     int N, T, Hl, Hkvl;
     int q_head0, kv_head0;
     float scale_log2;      // softmax scale * log2(e)
-    uint32_t *status;
+    int items;             // work items: ceil(T / 2) tile pairs x Hl heads
+    uint32_t *status;      // [0] status word, [1] work counter (both zeroed before the launch)
     uint64_t wait_limit_ns;
     uint32_t debug_flags;   // bit 0: CTA 0 waits on a barrier nobody arrives on (tests the timeout path)
 };
+
+// One work item: the tile pair q_order[idx / Hl] of head idx % Hl.
+struct FwdItem {
+    int h, kvh, tA, tB;
+    bool hasB;
+    int j0;        // first key tile of the union of both tiles' ranges
+    int nA;        // key tiles of A: union steps [0, nA)
+    int bstart;    // key tiles of B: union steps [bstart, n_union)
+    int nB;
+    int n_union;
+};
+
+__device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
+{
+    FwdItem it;
+    const int pair = p.q_order[idx / p.Hl];
+    it.h = idx % p.Hl;
+    it.kvh = it.h / (p.Hl / p.Hkvl);
+    it.tA = 2 * pair;
+    it.tB = 2 * pair + 1;
+    it.hasB = it.tB < p.T;
+    it.j0 = p.tile_lo[it.tA] / kTileN;
+    it.nA = it.tA - it.j0 + 1;
+    const int loB = it.hasB ? p.tile_lo[it.tB] / kTileN : 0;
+    it.bstart = it.hasB ? loB - it.j0 : 0;
+    it.nB = it.hasB ? it.tB - loB + 1 : 0;
+    it.n_union = it.hasB ? it.tB - it.j0 + 1 : it.nA;
+    return it;
+}
 
 template <int D>
 struct FwdCfg {
@@ -89,8 +126,8 @@ struct FwdCfg {
     static constexpr int OFF_K = 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
-    static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 1;
-    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;   // + alignment slack
+    static constexpr int NBAR = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 2 + 2 + 1 + 1;
+    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 16 + 1024;   // + item ring, alignment slack
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kTileM, kTileN, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kTileM, D, false, true);
     // tensor-memory columns: S / P of tile x at ts_col(x), O of tile x at to_col(x)
@@ -111,37 +148,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint8_t *sV = smem + C::OFF_V;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars;                 // [2]
-    uint64_t *k_full = bars + 2;             // [KST]
+    uint64_t *q_empty = bars + 2;            // [2] the last S of an item has read Q_x
+    uint64_t *k_full = bars + 4;             // [KST]
     uint64_t *k_empty = k_full + C::KST;
     uint64_t *v_full = k_empty + C::KST;     // [VST]
     uint64_t *v_empty = v_full + C::VST;
     uint64_t *s_full = v_empty + C::VST;     // [2] per tile
     uint64_t *p_full = s_full + 2;           // [2] per tile
     uint64_t *o_done = p_full + 2;           // [2] per tile
-    uint64_t *mma_done = o_done + 2;
+    uint64_t *item_full = o_done + 2;        // [2] item ring slot written
+    uint64_t *item_empty = item_full + 2;    // [2] item ring slot read by every consumer
+    uint64_t *mma_done = item_empty + 2;
     uint64_t *never = mma_done + 1;          // never arrived on (timeout test only)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(never + 1);
+    volatile int *item_ring = reinterpret_cast<volatile int *>(tmem_holder + 4);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- work item: a pair of query tiles, heaviest pairs first
-    const int item = blockIdx.x;
-    const int pair = p.q_order[item / p.Hl];
-    const int h = item % p.Hl;
-    const int kvh = h / (p.Hl / p.Hkvl);
-    const int tA = 2 * pair, tB = 2 * pair + 1;
-    const bool hasB = tB < p.T;
-    const int j0 = p.tile_lo[tA] / kTileN;                 // first key tile of the union
-    const int nA = tA - j0 + 1;                            // key tiles of A: union [0, nA)
-    const int loB = hasB ? p.tile_lo[tB] / kTileN : 0;
-    const int bstart = hasB ? loB - j0 : 0;                // key tiles of B: union [bstart, n_union)
-    const int nB = hasB ? tB - loB + 1 : 0;
-    const int n_union = hasB ? tB - j0 + 1 : nA;
+    // consumers of every ring slot: MMA warp (1), V producer (1), both softmax warpgroups (256)
+    constexpr uint32_t kItemConsumers = 2 + 256;
 
     if (threadIdx.x == 0) {
-        mbar_init(&q_full[0], 1);
-        mbar_init(&q_full[1], 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&q_full[x], 1);
+            mbar_init(&q_empty[x], 1);
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 128);
+            mbar_init(&o_done[x], 1);
+            mbar_init(&item_full[x], 1);
+            mbar_init(&item_empty[x], kItemConsumers);
+        }
         for (int s = 0; s < C::KST; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -149,11 +185,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int s = 0; s < C::VST; ++s) {
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
-        }
-        for (int x = 0; x < 2; ++x) {
-            mbar_init(&s_full[x], 1);
-            mbar_init(&p_full[x], 128);
-            mbar_init(&o_done[x], 1);
         }
         mbar_init(mma_done, 1);
         mbar_init(never, 1);
@@ -171,37 +202,62 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // A CTA that starts after another one has timed out skips its work.
     WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
 
+    // Consumer side of the item ring: the n-th item of this CTA (-1: no more work).
+    auto take_item = [&](int n, bool warp_wide) -> int {
+        const int slot = n & 1;
+        const bool ok = warp_wide ? mbar_wait_warp(&item_full[slot], (n >> 1) & 1, wc)
+                                  : mbar_wait(&item_full[slot], (n >> 1) & 1, wc);
+        if (!ok) return -1;
+        return item_ring[slot];
+    };
+
     if (warp >= 8) {
     setmaxnreg_dec<kControlRegs>();
     if (warp == kProducerWarp) {
-        // ================================================================ producer
+        // ================================================================ items, Q and K producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
-            for (int x = 0; x < (hasB ? 2 : 1); ++x) {
-                mbar_arrive_expect_tx(&q_full[x], C::TILE_BYTES);
-#pragma unroll
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_3d(sQ + x * C::TILE_BYTES + a * C::ATOM_BYTES, &tmQ, &q_full[x], a * C::AW,
-                                p.q_head0 + h, (x == 0 ? tA : tB) * kTileM);
-            }
+            int kcount = 0;                  // K tiles loaded so far (ring position)
+            int qcount[2] = {0, 0};          // Q_x tiles loaded so far
             int last_use[C::KST];
 #pragma unroll
             for (int s = 0; s < C::KST; ++s) last_use[s] = -1;
-            for (int j = 0; j < n_union; ++j) {
-                const int s = j % C::KST, u = j / C::KST;
-                if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) break;
-                mbar_arrive_expect_tx(&k_full[s], C::TILE_BYTES);
+            for (int n = 0;; ++n) {
+                const int slot = n & 1;
+                if (n >= 2 && !mbar_wait(&item_empty[slot], ((n >> 1) - 1) & 1, wc)) break;
+                int idx = static_cast<int>(atomicAdd(p.status + 1, 1u));
+                if (idx >= p.items) idx = -1;
+                item_ring[slot] = idx;
+                mbar_arrive(&item_full[slot]);
+                if (idx < 0) break;
+                const FwdItem w = decode_item(p, idx);
+                bool ok = true;
+                for (int x = 0; x < (w.hasB ? 2 : 1); ++x) {
+                    if (qcount[x] > 0 && !mbar_wait(&q_empty[x], (qcount[x] - 1) & 1, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&q_full[x], C::TILE_BYTES);
 #pragma unroll
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmK, &k_full[s], a * C::AW,
-                                p.kv_head0 + kvh, (j0 + j) * kTileN);
-                last_use[s] = u;
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_load_3d(sQ + x * C::TILE_BYTES + a * C::ATOM_BYTES, &tmQ, &q_full[x], a * C::AW,
+                                    p.q_head0 + w.h, (x == 0 ? w.tA : w.tB) * kTileM);
+                    ++qcount[x];
+                }
+                for (int j = 0; ok && j < w.n_union; ++j, ++kcount) {
+                    const int s = kcount % C::KST, u = kcount / C::KST;
+                    if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&k_full[s], C::TILE_BYTES);
+#pragma unroll
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmK, &k_full[s], a * C::AW,
+                                    p.kv_head0 + w.kvh, (w.j0 + j) * kTileN);
+                    last_use[s] = u;
+                }
+                if (!ok) break;
             }
             // Never leave the CTA with bulk copies still landing in its shared memory.
             WaitCtx drain{p.wait_limit_ns, p.status, false};
-            mbar_wait(&q_full[0], 0, drain);
-            if (hasB) mbar_wait(&q_full[1], 0, drain);
+            for (int x = 0; x < 2; ++x)
+                if (qcount[x] > 0) mbar_wait(&q_full[x], (qcount[x] - 1) & 1, drain);
             for (int s = 0; s < C::KST; ++s)
                 if (last_use[s] >= 0) mbar_wait(&k_full[s], last_use[s] & 1, drain);
         }
@@ -209,18 +265,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ================================================================ V producer
         if (lane == 0) {
             prefetch_tmap(&tmV);
+            int vcount = 0;
             int last_use[C::VST];
 #pragma unroll
             for (int s = 0; s < C::VST; ++s) last_use[s] = -1;
-            for (int j = 0; j < n_union; ++j) {
-                const int s = j % C::VST, u = j / C::VST;
-                if (u > 0 && !mbar_wait(&v_empty[s], (u - 1) & 1, wc)) break;
-                mbar_arrive_expect_tx(&v_full[s], C::TILE_BYTES);
+            for (int n = 0;; ++n) {
+                const int idx = take_item(n, false);
+                mbar_arrive(&item_empty[n & 1]);
+                if (idx < 0) break;
+                const FwdItem w = decode_item(p, idx);
+                bool ok = true;
+                for (int j = 0; j < w.n_union; ++j, ++vcount) {
+                    const int s = vcount % C::VST, u = vcount / C::VST;
+                    if (u > 0 && !mbar_wait(&v_empty[s], (u - 1) & 1, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&v_full[s], C::TILE_BYTES);
 #pragma unroll
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmV, &v_full[s], a * C::AW,
-                                p.kv_head0 + kvh, (j0 + j) * kTileN);
-                last_use[s] = u;
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_load_3d(sV + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmV, &v_full[s], a * C::AW,
+                                    p.kv_head0 + w.kvh, (w.j0 + j) * kTileN);
+                    last_use[s] = u;
+                }
+                if (!ok) break;
             }
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             for (int s = 0; s < C::VST; ++s)
@@ -230,206 +295,236 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ================================================================ MMA issuer
         // The whole warp runs the loop; one elected lane issues each tcgen05
         // instruction (faster than issuing from a one-lane branch).
-        {
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-            // S_x(it) = Q_x K_j^T, K-major operands, 16-element K steps
-            auto issue_s = [&](int x, int s) {
-                constexpr int steps = C::SW / 32;
+        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+        // S_x = Q_x K^T, K-major operands, 16-element K steps
+        // (descriptor of step kk = descriptor of step 0 + the step's byte offset >> 4)
+        auto issue_s = [&](int x, int s) {
+            constexpr int steps = C::SW / 32;
+            const uint64_t ad = smem_desc(aQ + x * C::TILE_BYTES, 16, 8 * C::SW, C::SWZ);
+            const uint64_t bd = smem_desc(aK + s * C::TILE_BYTES, 16, 8 * C::SW, C::SWZ);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk / steps) * C::ATOM_BYTES + (kk % steps) * 32;
-                    const uint64_t ad = smem_desc(aQ + x * C::TILE_BYTES + koff, 16, 8 * C::SW, C::SWZ);
-                    const uint64_t bd = smem_desc(aK + s * C::TILE_BYTES + koff, 16, 8 * C::SW, C::SWZ);
-                    umma_ss_elect(tbase + C::ts_col(x), ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-                }
-                umma_commit_elect(&s_full[x]);
-            };
-            // O_x += P_x V_j, P from tensor memory (8 columns per 16 keys)
-            auto issue_pv = [&](int x, int s, bool first) {
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = ((kk / steps) * C::ATOM_BYTES + (kk % steps) * 32) >> 4;
+                umma_ss_elect_off(tbase + C::ts_col(x), ad, koff, bd, koff, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            umma_commit_elect(&s_full[x]);
+        };
+        // O_x += P_x V, P from tensor memory (8 columns per 16 keys)
+        auto issue_pv = [&](int x, int s, bool first) {
+            const uint64_t bd = smem_desc(aV + s * C::TILE_BYTES, C::ATOM_BYTES, 8 * C::SW, C::SWZ);
 #pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk) {
-                    const uint64_t bd = smem_desc(aV + s * C::TILE_BYTES + kk * 16 * C::SW, C::ATOM_BYTES,
-                                                  8 * C::SW, C::SWZ);
-                    umma_ts_elect(tbase + C::to_col(x), tbase + C::ts_col(x) + kk * 8, bd, C::IDESC_PV,
-                                  (!first || kk > 0) ? 1u : 0u);
-                }
-            };
-            bool ok = mbar_wait_warp(&q_full[0], 0, wc);
-            if (ok && hasB) ok = mbar_wait_warp(&q_full[1], 0, wc);
-            for (int j = 0; ok && j <= n_union; ++j) {
-                const int s = j % C::KST, u = j / C::KST;                            // K stage of key tile j
-                const int sp = (j - 1 + C::VST) % C::VST, up = (j - 1) / C::VST;   // V stage of key tile j-1
-                const bool have_j = j < n_union;
-                const bool pvA = (j - 1 >= 0) && (j - 1 < nA);
-                const bool sA = have_j && j < nA;
-                const int jb = j - bstart;
-                const bool pvB = hasB && (jb - 1 >= 0) && (jb - 1 < nB);
-                const bool sB = hasB && have_j && jb >= 0 && jb < nB;
+            for (int kk = 0; kk < kTileN / 16; ++kk)
+                umma_ts_elect_off(tbase + C::to_col(x), tbase + C::ts_col(x) + kk * 8, bd, (kk * 16 * C::SW) >> 4,
+                                  C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+        };
+        int kbase = 0, vbase = 0;            // K / V tiles consumed by earlier items
+        int pbase[2] = {0, 0};               // P tiles of each tile slot consumed by earlier items
+        int qcount[2] = {0, 0};
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int idx = take_item(n, true);
+            if (lane == 0) mbar_arrive(&item_empty[n & 1]);
+            __syncwarp();
+            if (idx < 0) break;
+            const FwdItem w = decode_item(p, idx);
+            ok = mbar_wait_warp(&q_full[0], qcount[0] & 1, wc);
+            if (ok && w.hasB) ok = mbar_wait_warp(&q_full[1], qcount[1] & 1, wc);
+            for (int j = 0; ok && j <= w.n_union; ++j) {
+                const int gk = kbase + j, gv = vbase + j - 1;   // ring positions of K_j and V_(j-1)
+                const int s = gk % C::KST, u = gk / C::KST;
+                const int sp = (gv + C::VST) % C::VST, up = gv / C::VST;
+                const bool have_j = j < w.n_union;
+                const bool pvA = (j - 1 >= 0) && (j - 1 < w.nA);
+                const bool sA = have_j && j < w.nA;
+                const int jb = j - w.bstart;
+                const bool pvB = w.hasB && (jb - 1 >= 0) && (jb - 1 < w.nB);
+                const bool sB = w.hasB && have_j && jb >= 0 && jb < w.nB;
                 if ((pvA || pvB) && !mbar_wait_warp(&v_full[sp], up & 1, wc)) { ok = false; break; }
                 if ((sA || sB) && !mbar_wait_warp(&k_full[s], u & 1, wc)) { ok = false; break; }
                 // tile A
                 if (pvA) {
-                    if (!mbar_wait_warp(&p_full[0], (j - 1) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait_warp(&p_full[0], (pbase[0] + j - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(0, sp, j - 1 == 0);
-                    if (j - 1 == nA - 1) umma_commit_elect(&o_done[0]);
+                    if (j - 1 == w.nA - 1) umma_commit_elect(&o_done[0]);
                 }
                 if (sA) {
                     tc_fence_after();
                     issue_s(0, s);
+                    if (j == w.nA - 1) umma_commit_elect(&q_empty[0]);
                 }
                 // tile B
                 if (pvB) {
-                    if (!mbar_wait_warp(&p_full[1], (jb - 1) & 1, wc)) { ok = false; break; }
+                    if (!mbar_wait_warp(&p_full[1], (pbase[1] + jb - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(1, sp, jb - 1 == 0);
-                    if (jb - 1 == nB - 1) umma_commit_elect(&o_done[1]);
+                    if (jb - 1 == w.nB - 1) umma_commit_elect(&o_done[1]);
                 }
                 if (sB) {
                     tc_fence_after();
                     issue_s(1, s);
+                    if (jb == w.nB - 1) umma_commit_elect(&q_empty[1]);
                 }
                 if (sA || sB) umma_commit_elect(&k_empty[s]);
                 if (pvA || pvB) umma_commit_elect(&v_empty[sp]);
             }
-            umma_commit_elect(mma_done);
-            WaitCtx drain{p.wait_limit_ns, p.status, false};
-            mbar_wait(mma_done, 0, drain);
+            kbase += w.n_union;
+            vbase += w.n_union;
+            pbase[0] += w.nA;
+            pbase[1] += w.nB;
+            ++qcount[0];
+            if (w.hasB) ++qcount[1];
         }
+        umma_commit_elect(mma_done);
+        WaitCtx drain{p.wait_limit_ns, p.status, false};
+        mbar_wait(mma_done, 0, drain);
     }
     } else {
         setmaxnreg_inc<kSoftmaxRegs>();
         // ================================================================ softmax warpgroups
         const int x = warp >> 2;                                   // 0: tile A, 1: tile B
-        const int n_it = x == 0 ? nA : nB;
-        const int first_union = x == 0 ? 0 : bstart;
         const int r = threadIdx.x & 127;                           // row within the tile == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tbase + C::ts_col(x) + lane_off;
         const uint32_t tO = tbase + C::to_col(x) + lane_off;
-        const int i = (x == 0 ? tA : tB) * kTileM + r;
-        const bool valid = i < p.N;
-        const int lo = valid ? p.doc_start[i] : i;
-        const int hi = i;
         const float sl2 = p.scale_log2;
-        float ms = -CUDART_INF_F;   // exponent offset in use (scaled log2 units)
-        float l = 0.f;
+        int sbase = 0;      // S tiles of this slot consumed by earlier items
+        int ocount = 0;     // items finished by this slot
         bool ok = true;
         if ((p.debug_flags & 1u) && blockIdx.x == 0 && x == 0) ok = mbar_wait(never, 0, wc);   // runs out
-        for (int it = 0; it < n_it; ++it) {
-            if (!mbar_wait(&s_full[x], it & 1, wc)) { ok = false; break; }
-            tc_fence_after();
-            float s[kTileN];
-            {
-                uint32_t raw0[64], raw1[64];
-                tmem_ld64(tS, raw0);
-                tmem_ld64(tS + 64, raw1);
-                tmem_ld_wait();
+        for (int n = 0; ok; ++n) {
+            const int idx = take_item(n, false);
+            mbar_arrive(&item_empty[n & 1]);
+            if (idx < 0) break;
+            const FwdItem w = decode_item(p, idx);
+            const int n_it = x == 0 ? w.nA : w.nB;
+            if (n_it == 0) continue;
+            const int first_union = x == 0 ? 0 : w.bstart;
+            const int i = (x == 0 ? w.tA : w.tB) * kTileM + r;
+            const bool valid = i < p.N;
+            const int lo = valid ? p.doc_start[i] : i;
+            const int hi = i;
+            float ms = -CUDART_INF_F;   // exponent offset in use (scaled log2 units)
+            float l = 0.f;
+            for (int it = 0; it < n_it; ++it) {
+                if (!mbar_wait(&s_full[x], (sbase + it) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                float s[kTileN];
+                {
+                    uint32_t raw0[64], raw1[64];
+                    tmem_ld64(tS, raw0);
+                    tmem_ld64(tS + 64, raw1);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    s[e] = __uint_as_float(raw0[e]);
-                    s[64 + e] = __uint_as_float(raw1[e]);
+                    for (int e = 0; e < 64; ++e) {
+                        s[e] = __uint_as_float(raw0[e]);
+                        s[64 + e] = __uint_as_float(raw1[e]);
+                    }
                 }
-            }
-            const int c0 = (j0 + first_union + it) * kTileN;
-            // This row may see key columns [cl, ch) of the tile. A row that sees
-            // none (its document starts in a later key tile: a tile straddling
-            // a document boundary) is zeroed through its exponent offset below;
-            // only rows cut inside the tile need a per-column mask.
-            const int cl = lo - c0, ch = hi - c0 + 1;
-            const bool row_out = cl >= kTileN;
-            if (__any_sync(0xffffffffu, !row_out && (cl > 0 || ch < kTileN))) {
-                // 32-column chunks valid for the whole warp are skipped; the
-                // others select column by column, branch-free.
+                const int c0 = (w.j0 + first_union + it) * kTileN;
+                // This row may see key columns [cl, ch) of the tile. A row that sees
+                // none (its document starts in a later key tile: a tile straddling
+                // a document boundary) is zeroed through its exponent offset below;
+                // only rows cut inside the tile need a per-column mask.
+                const int cl = lo - c0, ch = hi - c0 + 1;
+                const bool row_out = cl >= kTileN;
+                if (__any_sync(0xffffffffu, !row_out && (cl > 0 || ch < kTileN))) {
+                    // 32-column chunks valid for the whole warp are skipped; the
+                    // others select column by column, branch-free.
 #pragma unroll
-                for (int k = 0; k < kTileN / 32; ++k) {
-                    if (!__all_sync(0xffffffffu, cl <= 32 * k && ch >= 32 * k + 32)) {
+                    for (int k = 0; k < kTileN / 32; ++k) {
+                        if (!__all_sync(0xffffffffu, cl <= 32 * k && ch >= 32 * k + 32)) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int c = 32 * k + e;
-                            s[c] = (c >= cl && c < ch) ? s[c] : -CUDART_INF_F;
+                            for (int e = 0; e < 32; ++e) {
+                                const int c = 32 * k + e;
+                                s[c] = (c >= cl && c < ch) ? s[c] : -CUDART_INF_F;
+                            }
                         }
                     }
                 }
-            }
-            // row max: 4 independent chains of 3-input max
-            float mx[4] = {s[0], s[1], s[2], s[3]};
+                // row max: 4 independent chains of 3-input max
+                float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 4; c < kTileN; c += 8)
+                for (int c = 4; c < kTileN; c += 8)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[c + e], s[c + 4 + e]);
-            const float mt = row_out ? -CUDART_INF_F : max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-            const float mt_s = mt * sl2;
-            const bool resc = mt_s > ms + 8.0f;
-            float alpha = 1.f;
-            if (resc) {
-                alpha = ex2_approx(ms - mt_s);
-                ms = mt_s;
-                l *= alpha;
-            }
-            if (it > 0 && __any_sync(0xffffffffu, resc)) {
-                // O holds the previous tiles' sum in the old units. PV_x(it-1)
-                // was issued before S_x(it), so it has completed.
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t raw[32];
-                    tmem_ld32(tO + c * 32, raw);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-                    tmem_st32(tO + c * 32, raw);
+                    for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[c + e], s[c + 4 + e]);
+                const float mt = row_out ? -CUDART_INF_F : max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+                const float mt_s = mt * sl2;
+                const bool resc = mt_s > ms + 8.0f;
+                float alpha = 1.f;
+                if (resc) {
+                    alpha = ex2_approx(ms - mt_s);
+                    ms = mt_s;
+                    l *= alpha;
                 }
-            }
-            // offset +inf turns every exponent of an all-masked row into exp2(-inf)
-            const float moff = row_out ? CUDART_INF_F : ((ms == -CUDART_INF_F) ? 0.f : ms);
-            // P = exp2(s * scale*log2(e) - offset): the argument two columns at a
-            // time (packed FMA), the exponential on the SFU, the row sum two
-            // columns at a time (packed add, 4 independent accumulator pairs).
-            float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[64];
+                if (it > 0 && __any_sync(0xffffffffu, resc)) {
+                    // O holds the previous tiles' sum in the old units. PV_x(it-1)
+                    // was issued before S_x(it), so it has completed.
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                float x0, x1;
-                fma2_bcast(x0, x1, s[2 * e], s[2 * e + 1], sl2, -moff);
-                // 3 column pairs in 8 take the FMA-pipe exponential, the rest the SFU
-                float e0, e1;
-                if ((e & 7) < kEmuPairs) {
-                    ex2_poly2(e0, e1, x0, x1);
-                } else {
-                    e0 = ex2_approx(x0);
-                    e1 = ex2_approx(x1);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t raw[32];
+                        tmem_ld32(tO + c * 32, raw);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+                        tmem_st32(tO + c * 32, raw);
+                    }
                 }
-                add2_acc(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], e0, e1);
-                pk[e] = pack_bf16x2(e0, e1);
+                // offset +inf turns every exponent of an all-masked row into exp2(-inf)
+                const float moff = row_out ? CUDART_INF_F : ((ms == -CUDART_INF_F) ? 0.f : ms);
+                // P = exp2(s * scale*log2(e) - offset): the argument two columns at a
+                // time (packed FMA), the exponential on the SFU, the row sum two
+                // columns at a time (packed add, 4 independent accumulator pairs).
+                float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                uint32_t pk[64];
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    float x0, x1;
+                    fma2_bcast(x0, x1, s[2 * e], s[2 * e + 1], sl2, -moff);
+                    // 3 column pairs in 8 take the FMA-pipe exponential, the rest the SFU
+                    float e0, e1;
+                    if ((e & 7) < kEmuPairs) {
+                        ex2_poly2(e0, e1, x0, x1);
+                    } else {
+                        e0 = ex2_approx(x0);
+                        e1 = ex2_approx(x1);
+                    }
+                    add2_acc(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], e0, e1);
+                    pk[e] = pack_bf16x2(e0, e1);
+                }
+                tmem_st64(tS, pk);   // P overwrites the first 64 columns of S
+                l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&p_full[x]);
             }
-            tmem_st64(tS, pk);   // P overwrites the first 64 columns of S
-            l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&p_full[x]);
-        }
-        // ---- epilogue: O / l -> bf16, LSE
-        if (ok && n_it > 0 && mbar_wait(&o_done[x], 0, wc)) {
+            sbase += n_it;
+            // ---- epilogue: O / l -> bf16, LSE. The next item's first PV into O_x
+            // waits for this slot's next P, which comes after these reads.
+            if (!ok || !mbar_wait(&o_done[x], ocount & 1, wc)) { ok = false; break; }
+            ++ocount;
             tc_fence_after();
             const float inv_l = 1.f / l;
             __nv_bfloat16 *orow = p.o + static_cast<int64_t>(i) * p.o_row_elems +
-                                  static_cast<int64_t>(p.o_head0 + h) * D;
+                                  static_cast<int64_t>(p.o_head0 + w.h) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t raw[32];
                 tmem_ld32(tO + c * 32, raw);
                 tmem_ld_wait();
-                uint32_t w[16];
+                uint32_t wv[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l, __uint_as_float(raw[2 * e + 1]) * inv_l);
+                    wv[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l, __uint_as_float(raw[2 * e + 1]) * inv_l);
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
                 }
             }
-            if (valid) p.lse[static_cast<int64_t>(h) * p.N + i] = (ms + __log2f(l)) * 0.69314718055994530942f;
+            if (valid) p.lse[static_cast<int64_t>(w.h) * p.N + i] = (ms + __log2f(l)) * 0.69314718055994530942f;
+            tc_fence_before();
         }
     }
 
@@ -469,20 +564,25 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.kv_head0 = a.kv_head0;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.status = reinterpret_cast<uint32_t *>(const_cast<char *>(a.ws) + a.L.status);
+    p.items = static_cast<int>(ceil_div(p.T, 2) * a.Hl);
     p.wait_limit_ns = a.wait_limit_ns;
     p.debug_flags = a.debug_flags;
     static bool attr_set[64] = {};
+    static int sm_count[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
         cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const int64_t pairs = ceil_div(p.T, 2);
-    const int64_t items = pairs * a.Hl;
-    attn_fwd_kernel<D><<<static_cast<unsigned>(items), kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    // persistent: one CTA per SM (each needs a whole SM's tensor memory)
+    const int sms = (dev < 64 && sm_count[dev] > 0) ? sm_count[dev] : 148;
+    const int grid = p.items < sms ? p.items : sms;
+    attn_fwd_kernel<D><<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 

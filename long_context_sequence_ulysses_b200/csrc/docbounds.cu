@@ -37,7 +37,10 @@ __global__ void __launch_bounds__(kScanBlock) doc_scan_kernel(const int32_t *__r
                                                              int32_t *__restrict__ block_agg,
                                                              uint32_t *__restrict__ status)
 {
-    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;   // fresh status for this call
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        status[0] = 0u;   // fresh status for this call
+        status[1] = 0u;   // work counter of the persistent forward kernel
+    }
     __shared__ int warp_max[kScanBlock / 32];
     const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
     int v = (i < N && pos[i] == 0) ? static_cast<int>(i) : 0;

@@ -17,7 +17,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace layout (every section 256-byte aligned):
-//   status     uint32 [64]        status word (bit 0: a bounded wait ran out)
+//   status     uint32 [64]        [0] status word (bit 0: a bounded wait ran out),
+//                                 [1] work counter of the persistent forward kernel
 //   doc_start  int32  [N]         first token of the row's document
 //   tile_lo    int32  [T]         doc_start of the first row of each 128-row tile
 //   q_order    int32  [T]         forward: pairs of query tiles (2u, 2u+1), heaviest
