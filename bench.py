@@ -51,9 +51,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_sha() -> str:
+# Sources a kernel's DRAM traffic depends on (its own file and the shared headers).
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("attn_fwd.cu", "ptx.cuh", "ulysses_internal.cuh"),
+    "attn_bwd_dkdv_kernel": ("attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh"),
+    "attn_bwd_dq_kernel": ("attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in ("attn_fwd.cu", "attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh"):
+    for name in KERNEL_SOURCES.get(kernel, ("attn_fwd.cu", "attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh")):
         p = os.path.join(ROOT, "long_context_sequence_ulysses_b200", "csrc", name)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -62,10 +70,10 @@ def kernel_source_sha() -> str:
 
 def lookup_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, valid only while the
-    kernel sources are unchanged since the capture."""
+    kernel's sources are unchanged since the capture."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel)
     for ln in open(TRAFFIC_FILE):
         ln = ln.strip()
         if not ln or ln.startswith("#"):
