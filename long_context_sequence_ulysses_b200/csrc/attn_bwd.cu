@@ -18,7 +18,11 @@
 //       S^T = K Q^T, dP^T = V dO^T       (SS MMA, M = keys, N = queries)
 //       P^T, dS^T -> bf16 into the first 64 columns of S^T / dP^T in TMEM
 //       dV += P^T dO, dK += dS^T Q      (TS MMA, dO / Q read MN-major)
-//     so the group reduction happens in the accumulator.
+//     so the group reduction happens in the accumulator. The element-wise
+//     step runs in two phases so that the tensor core always has work: once
+//     P^T(i) is stored, dV(i) and S^T(i+1) run while dS^T(i) is computed
+//     (from the bf16 P^T kept in registers); once dS^T(i) is stored, dK(i)
+//     and dP^T(i+1) run while P^T(i+1) is computed.
 //  3. dQ: one CTA per (query tile, head) loops over its key tiles:
 //       S = Q K^T, dP = dO V^T -> dS (bf16, into S's columns) -> dQ += dS K.
 #include "ptx.cuh"
@@ -31,8 +35,17 @@ namespace uly {
 
 namespace {
 
-constexpr int kBwdThreads = 256;
-constexpr int kComputeWarp0 = 4;   // warps 4..7: the compute warpgroup (TMEM lanes 0..127)
+// Warps 0..3: producers and the MMA issuer; warps 4..11: the element-wise
+// step. Compute warp w handles the 32 TMEM lanes (rows) of quarter w % 4 and
+// half (w - 4) / 4 of the 128 columns: the special-function unit and the
+// latency of each phase are shared by two warps per SM sub-partition. Each half
+// writes its bf16 results to its own 32-column region (half 0: columns 0..31,
+// half 1: columns 64..95 of the tile's 128), so neither overwrites columns
+// the other still has to read; the TS MMAs take K steps 4..7 from +64.
+constexpr int kBwdThreads = 384;
+constexpr int kComputeWarp0 = 4;
+// Column pairs (out of every 8) whose exponentials run on the FMA pipe.
+constexpr int kBwdEmuPairs = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -72,13 +85,19 @@ struct BwdCfg {
     static constexpr int KV_OFF_ROW = KV_OFF_DO + NST * TILE_BYTES;
     static constexpr int KV_OFF_BAR = KV_OFF_ROW + NST * 2 * 512;
     static constexpr int KV_SMEM = KV_OFF_BAR + 16 * 8 + 16 + 1024;
-    // dQ kernel shared memory: Q, dO, then NST stages of {K, V}, then barriers.
+    // dQ kernel shared memory: Q, dO, then QKST stages of K and QVST of V,
+    // then barriers. S runs two key tiles ahead of dQ, so a K tile is needed
+    // about two steps after its slot frees only with a third K stage; a V
+    // tile is read once, one step ahead.
+    static constexpr int QKST = (D == 128) ? 3 : 4;
+    static constexpr int QVST = (D == 128) ? 2 : 4;
     static constexpr int Q_OFF_Q = 0;
     static constexpr int Q_OFF_DO = TILE_BYTES;
     static constexpr int Q_OFF_K = 2 * TILE_BYTES;
-    static constexpr int Q_OFF_V = Q_OFF_K + NST * TILE_BYTES;
-    static constexpr int Q_OFF_BAR = Q_OFF_V + NST * TILE_BYTES;
-    static constexpr int Q_SMEM = Q_OFF_BAR + 16 * 8 + 16 + 1024;
+    static constexpr int Q_OFF_V = Q_OFF_K + QKST * TILE_BYTES;
+    static constexpr int Q_OFF_BAR = Q_OFF_V + QVST * TILE_BYTES;
+    static constexpr int Q_SMEM = Q_OFF_BAR + 24 * 8 + 16 + 1024;
+    static constexpr uint32_t T_S2 = 384;   // dQ kernel: second S buffer
 };
 
 __device__ __forceinline__ float dot8_bf16(const uint4 &a, const uint4 &b)
@@ -130,6 +149,10 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
         : "memory");
 }
 
+// Column of the bf16 operand packed in tensor memory for K step kk (16 rows
+// of the 128, two per column): half 0 wrote columns 0..31, half 1 64..95.
+__device__ __forceinline__ uint32_t pcol(int kk) { return static_cast<uint32_t>(kk * 8 + (kk >= 4 ? 32 : 0)); }
+
 // K-major SS descriptors for a 16-element K step kk of a 128-row tile.
 template <int D>
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int kk)
@@ -176,9 +199,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *kv_full = bars;
     uint64_t *qdo_full = bars + 1;            // [NST]
     uint64_t *qdo_empty = qdo_full + C::NST;  // [NST]
-    uint64_t *s_full = qdo_empty + C::NST;
-    uint64_t *ds_full = s_full + 1;
-    uint64_t *acc_done = ds_full + 1;
+    uint64_t *s_full = qdo_empty + C::NST;   // S^T(i) computed
+    uint64_t *ds_full = s_full + 1;           // dS^T(i) stored (256 arrivals)
+    uint64_t *dp_full = ds_full + 1;          // dP^T(i) computed
+    uint64_t *p_ready = dp_full + 1;          // P^T(i) stored (256 arrivals)
+    uint64_t *acc_done = p_ready + 1;
     uint64_t *mma_done = acc_done + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
 
@@ -198,7 +223,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&qdo_empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(ds_full, 128);
+        mbar_init(ds_full, 256);
+        mbar_init(dp_full, 1);
+        mbar_init(p_ready, 256);
         mbar_init(acc_done, 1);
         mbar_init(mma_done, 1);
         fence_mbar_init();
@@ -245,30 +272,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         {   // the whole warp runs the loop; elect.sync picks the issuing lane
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
             bool ok = mbar_wait_warp(kv_full, 0, wc);
+            auto issue_s = [&](int st) {   // S^T = K Q^T for the query tile in stage st
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_elect(tbase + C::T_S, kmajor_desc<D>(aK, kk), kmajor_desc<D>(aQ + st * C::TILE_BYTES, kk),
+                                  C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_commit_elect(s_full);
+            };
+            auto issue_dp = [&](int st) {   // dP^T = V dO^T
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_elect(tbase + C::T_DP, kmajor_desc<D>(aV, kk), kmajor_desc<D>(aDO + st * C::TILE_BYTES, kk),
+                                  C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_commit_elect(dp_full);
+            };
+            if (ok && n_it > 0) {
+                ok = mbar_wait_warp(&qdo_full[0], 0, wc);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0);
+                    issue_dp(0);
+                }
+            }
             for (int it = 0; ok && it < n_it; ++it) {
-                const int s = it % C::NST, u = it / C::NST;
-                if (!mbar_wait_warp(&qdo_full[s], u & 1, wc)) { ok = false; break; }
+                const int s = it % C::NST;
+                const int s1 = (it + 1) % C::NST, u1 = (it + 1) / C::NST;
+                const bool more = it + 1 < n_it;
+                if (!mbar_wait_warp(p_ready, it & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_elect(tbase + C::T_S, kmajor_desc<D>(aK, kk), kmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
-                            C::IDESC_SS, kk > 0 ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_elect(tbase + C::T_DP, kmajor_desc<D>(aV, kk), kmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
-                            C::IDESC_SS, kk > 0 ? 1u : 0u);
-                umma_commit_elect(s_full);
+                for (int kk = 0; kk < kTileM / 16; ++kk)   // dV += P^T dO
+                    umma_ts_elect(tbase + C::T_ACC0, tbase + C::T_S + pcol(kk), mnmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
+                                  C::IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+                // the next S^T overwrites P^T(it), which the dV products above read first
+                if (more) {
+                    if (!mbar_wait_warp(&qdo_full[s1], u1 & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_s(s1);
+                }
                 if (!mbar_wait_warp(ds_full, it & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kTileM / 16; ++kk) {
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts_elect(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aDO + s * C::TILE_BYTES, kk),
-                            C::IDESC_TS, acc);   // dV += P^T dO
-                    umma_ts_elect(tbase + C::T_ACC1, tbase + C::T_DP + kk * 8, mnmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
-                            C::IDESC_TS, acc);   // dK += dS^T Q
-                }
+                for (int kk = 0; kk < kTileM / 16; ++kk)   // dK += dS^T Q
+                    umma_ts_elect(tbase + C::T_ACC1, tbase + C::T_DP + pcol(kk), mnmajor_desc<D>(aQ + s * C::TILE_BYTES, kk),
+                                  C::IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
                 umma_commit_elect(&qdo_empty[s]);
+                if (more) issue_dp(s1);
             }
             if (ok) umma_commit_elect(acc_done);
             umma_commit_elect(mma_done);
@@ -276,9 +325,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(mma_done, 0, drain);
         }
     } else if (warp >= kComputeWarp0) {
-        // ------------------------------------------------ compute warpgroup: thread r owns key row r
-        const int r = threadIdx.x - kComputeWarp0 * 32;
-        const uint32_t lane_off = static_cast<uint32_t>((warp - kComputeWarp0) * 32) << 16;
+        // ------------------------------------------------ element-wise: thread = key row r, 64 query columns
+        const int quad = warp & 3, half = (warp - kComputeWarp0) >> 2;
+        const int r = quad * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int j = t * kTileN + r;
         // keys past N see no query; otherwise the queries of key j are [j, dend)
         int dend = j;
@@ -294,77 +344,90 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int s = it % C::NST, u = it / C::NST;
-            const int q0 = (qt0 + it % n_q) * kTileM;
+            const int q0 = (qt0 + it % n_q) * kTileM + half * 64;   // first query of this half
             if (!mbar_wait(s_full, it & 1, wc)) { ok = false; break; }
             if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const float *rl = sRow + (s * 2 + 0) * 128;   // -lse2 of the 128 queries
-            const float *rd = sRow + (s * 2 + 1) * 128;   // delta of the 128 queries
-            const bool need_mask = (q0 < j) || (q0 + kTileM - 1 >= dend);
-            const bool any_mask = __any_sync(0xffffffffu, need_mask);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sr[64], dr[64];
+            const float *rl = sRow + (s * 2 + 0) * 128 + half * 64;   // -lse2 of this half's queries
+            const float *rd = sRow + (s * 2 + 1) * 128 + half * 64;   // delta of this half's queries
+            const bool any_mask = __any_sync(0xffffffffu, (q0 < j) || (q0 + 63 >= dend));
+            // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns
+            uint32_t pp[32];
+            {
+                uint32_t sr[64];
                 tmem_ld64(tbase + C::T_S + lane_off + half * 64, sr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float2 nl = *reinterpret_cast<const float2 *>(rl + 2 * e);
+                    float x0, x1;
+                    fma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, nl.x, nl.y);
+                    if (any_mask) {
+                        const int qi = q0 + 2 * e;
+                        if (qi < j || qi >= dend) x0 = -CUDART_INF_F;
+                        if (qi + 1 < j || qi + 1 >= dend) x1 = -CUDART_INF_F;
+                    }
+                    float p0, p1;
+                    if ((e & 7) < kBwdEmuPairs) {
+                        ex2_poly2(p0, p1, x0, x1);
+                    } else {
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
+                    pp[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tbase + C::T_S + lane_off + half * 64, pp);   // P^T (queries packed in pairs)
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(p_ready);
+            // phase 2: dS^T = P^T (dP^T - D) from the bf16 P^T, bf16 into dP^T's columns
+            if (!mbar_wait(dp_full, it & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t dr[64];
                 tmem_ld64(tbase + C::T_DP + lane_off + half * 64, dr);
                 tmem_ld_wait();
-                uint32_t pp[32], dd[32];
+                uint32_t dd[32];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int c = half * 64 + 2 * e;   // columns c .. c+3
-                    const float4 nl = *reinterpret_cast<const float4 *>(rl + c);
-                    const float4 dl = *reinterpret_cast<const float4 *>(rd + c);
-                    float x[4], pv[4], t[4], dv[4];
-                    fma2(x[0], x[1], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, nl.x, nl.y);
-                    fma2(x[2], x[3], __uint_as_float(sr[2 * e + 2]), __uint_as_float(sr[2 * e + 3]), sl2, sl2, nl.z,
-                         nl.w);
-                    if (any_mask) {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int qi = q0 + c + k;
-                            if (qi < j || qi >= dend) x[k] = -CUDART_INF_F;
-                        }
-                    }
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) pv[k] = ex2_approx(x[k]);
-                    sub2(t[0], t[1], __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), dl.x, dl.y);
-                    sub2(t[2], t[3], __uint_as_float(dr[2 * e + 2]), __uint_as_float(dr[2 * e + 3]), dl.z, dl.w);
-                    mul2(dv[0], dv[1], pv[0], pv[1], t[0], t[1]);
-                    mul2(dv[2], dv[3], pv[2], pv[3], t[2], t[3]);
-                    pp[e] = pack_bf16x2(pv[0], pv[1]);
-                    pp[e + 1] = pack_bf16x2(pv[2], pv[3]);
-                    dd[e] = pack_bf16x2(dv[0], dv[1]);
-                    dd[e + 1] = pack_bf16x2(dv[2], dv[3]);
+                for (int e = 0; e < 32; ++e) {
+                    const float2 dl = *reinterpret_cast<const float2 *>(rd + 2 * e);
+                    const uint32_t pe = pp[e];
+                    float t0, t1, d0, d1;
+                    sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), dl.x, dl.y);
+                    mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
+                    dd[e] = pack_bf16x2(d0, d1);
                 }
-                tmem_st32(tbase + C::T_S + lane_off + half * 32, pp);    // P^T  (queries packed in pairs)
-                tmem_st32(tbase + C::T_DP + lane_off + half * 32, dd);   // dS^T
+                tmem_st32(tbase + C::T_DP + lane_off + half * 64, dd);   // dS^T
             }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(ds_full);
         }
+        // ---- epilogue: this half writes d columns [half * D/2, (half + 1) * D/2) of dV and dK
         if (ok && mbar_wait(acc_done, 0, wc)) {
             tc_fence_after();
             const bool valid = j < p.N;
-            __nv_bfloat16 *dv_row = p.dv + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D;
-            __nv_bfloat16 *dk_row = p.dk + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D;
+            __nv_bfloat16 *dv_row = p.dv + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + half * (D / 2);
+            __nv_bfloat16 *dk_row = p.dk + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + half * (D / 2);
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const float mul = which == 0 ? 1.f : p.scale;
                 __nv_bfloat16 *row = which == 0 ? dv_row : dk_row;
+                const uint32_t tacc = tbase + (which == 0 ? C::T_ACC0 : C::T_ACC1) + lane_off + half * (D / 2);
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    uint32_t raw[32];
-                    tmem_ld32(tbase + (which == 0 ? C::T_ACC0 : C::T_ACC1) + lane_off + c * 32, raw);
+                    uint32_t raw[16];
+                    tmem_ld16(tacc + c * 16, raw);
                     tmem_ld_wait();
-                    uint32_t w[16];
+                    uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
+                    for (int e = 0; e < 8; ++e)
                         w[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * mul, __uint_as_float(raw[2 * e + 1]) * mul);
                     if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(row + c * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                        uint4 *dst = reinterpret_cast<uint4 *>(row + c * 16);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     }
                 }
             }
@@ -393,10 +456,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *sV = smem + C::Q_OFF_V;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::Q_OFF_BAR);
     uint64_t *qdo_full = bars;
-    uint64_t *kv_full = bars + 1;           // [NST]
-    uint64_t *kv_empty = kv_full + C::NST;  // [NST]
-    uint64_t *s_full = kv_empty + C::NST;
-    uint64_t *ds_full = s_full + 1;
+    uint64_t *k_full = bars + 1;             // [QKST]
+    uint64_t *k_empty = k_full + C::QKST;    // [QKST] S(j) and dQ(j) have read K_j
+    uint64_t *v_full = k_empty + C::QKST;    // [QVST]
+    uint64_t *v_empty = v_full + C::QVST;    // [QVST] dP(j) has read V_j
+    uint64_t *s_full = v_empty + C::QVST;    // [2] S(j) computed into buffer j % 2
+    uint64_t *dp_full = s_full + 2;          // dP(j) computed
+    uint64_t *ds_full = dp_full + 1;         // dS(j) stored (256 arrivals)
     uint64_t *acc_done = ds_full + 1;
     uint64_t *mma_done = acc_done + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
@@ -411,12 +477,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(qdo_full, 1);
-        for (int s = 0; s < C::NST; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < C::QKST; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(ds_full, 128);
+        for (int s = 0; s < C::QVST; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(dp_full, 1);
+        mbar_init(ds_full, 256);
         mbar_init(acc_done, 1);
         mbar_init(mma_done, 1);
         fence_mbar_init();
@@ -432,50 +504,86 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
 
     if (warp == 0) {
+        // ------------------------------------------------ Q, dO and K producer
         if (lane == 0) {
             mbar_arrive_expect_tx(qdo_full, 2 * C::TILE_BYTES);
             tma_tile<D>(&tmQ, sQ, qdo_full, h, qt * kTileM);
             tma_tile<D>(&tmDO, sDO, qdo_full, h, qt * kTileM);
-            int last_use[C::NST];
+            int last_use[C::QKST];
 #pragma unroll
-            for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
+            for (int s = 0; s < C::QKST; ++s) last_use[s] = -1;
             for (int j = 0; j < n_kv; ++j) {
-                const int s = j % C::NST, u = j / C::NST;
-                if (u > 0 && !mbar_wait(&kv_empty[s], (u - 1) & 1, wc)) break;
-                mbar_arrive_expect_tx(&kv_full[s], 2 * C::TILE_BYTES);
-                tma_tile<D>(&tmK, sK + s * C::TILE_BYTES, &kv_full[s], kvh, (kt0 + j) * kTileN);
-                tma_tile<D>(&tmV, sV + s * C::TILE_BYTES, &kv_full[s], kvh, (kt0 + j) * kTileN);
+                const int s = j % C::QKST, u = j / C::QKST;
+                if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) break;
+                mbar_arrive_expect_tx(&k_full[s], C::TILE_BYTES);
+                tma_tile<D>(&tmK, sK + s * C::TILE_BYTES, &k_full[s], kvh, (kt0 + j) * kTileN);
                 last_use[s] = u;
             }
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(qdo_full, 0, drain);
-            for (int s = 0; s < C::NST; ++s)
-                if (last_use[s] >= 0) mbar_wait(&kv_full[s], last_use[s] & 1, drain);
+            for (int s = 0; s < C::QKST; ++s)
+                if (last_use[s] >= 0) mbar_wait(&k_full[s], last_use[s] & 1, drain);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------ V producer
+        if (lane == 0) {
+            int last_use[C::QVST];
+#pragma unroll
+            for (int s = 0; s < C::QVST; ++s) last_use[s] = -1;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j % C::QVST, u = j / C::QVST;
+                if (u > 0 && !mbar_wait(&v_empty[s], (u - 1) & 1, wc)) break;
+                mbar_arrive_expect_tx(&v_full[s], C::TILE_BYTES);
+                tma_tile<D>(&tmV, sV + s * C::TILE_BYTES, &v_full[s], kvh, (kt0 + j) * kTileN);
+                last_use[s] = u;
+            }
+            WaitCtx drain{p.wait_limit_ns, p.status, false};
+            for (int s = 0; s < C::QVST; ++s)
+                if (last_use[s] >= 0) mbar_wait(&v_full[s], last_use[s] & 1, drain);
         }
     } else if (warp == 1) {
         {   // the whole warp runs the loop; elect.sync picks the issuing lane
             const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
             bool ok = mbar_wait_warp(qdo_full, 0, wc);
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int s = j % C::NST, u = j / C::NST;
-                if (!mbar_wait_warp(&kv_full[s], u & 1, wc)) { ok = false; break; }
+            auto sbuf = [&](int jj) { return tbase + ((jj & 1) ? C::T_S2 : C::T_S); };
+            auto issue_s = [&](int jj) -> bool {   // S(jj) = Q K_jj^T into buffer jj % 2
+                const int s = jj % C::QKST;
+                if (!mbar_wait_warp(&k_full[s], (jj / C::QKST) & 1, wc)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss_elect(tbase + C::T_S, kmajor_desc<D>(aQ, kk), kmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
-                            C::IDESC_SS, kk > 0 ? 1u : 0u);
+                    umma_ss_elect(sbuf(jj), kmajor_desc<D>(aQ, kk), kmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
+                                  C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_commit_elect(&s_full[jj & 1]);
+                return true;
+            };
+            auto issue_dp = [&](int jj) -> bool {   // dP(jj) = dO V_jj^T
+                const int s = jj % C::QVST;
+                if (!mbar_wait_warp(&v_full[s], (jj / C::QVST) & 1, wc)) return false;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     umma_ss_elect(tbase + C::T_DP, kmajor_desc<D>(aDO, kk), kmajor_desc<D>(aV + s * C::TILE_BYTES, kk),
-                            C::IDESC_SS, kk > 0 ? 1u : 0u);
-                umma_commit_elect(s_full);
+                                  C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_commit_elect(dp_full);
+                umma_commit_elect(&v_empty[s]);
+                return true;
+            };
+            if (ok && n_kv > 0) ok = issue_s(0) && issue_dp(0);
+            if (ok && n_kv > 1) ok = issue_s(1);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j % C::QKST;
                 if (!mbar_wait_warp(ds_full, j & 1, wc)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTileN / 16; ++kk)
-                    umma_ts_elect(tbase + C::T_ACC0, tbase + C::T_S + kk * 8, mnmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
-                            C::IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);   // dQ += dS K
-                umma_commit_elect(&kv_empty[s]);
+                    umma_ts_elect(tbase + C::T_ACC0, sbuf(j) + pcol(kk), mnmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
+                                  C::IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);   // dQ += dS K
+                umma_commit_elect(&k_empty[s]);
+                // dP(j+1) overwrites dP(j), read by the element-wise step of j;
+                // S(j+2) overwrites dS(j), read by the products just issued
+                if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
+                if (j + 2 < n_kv && !issue_s(j + 2)) { ok = false; break; }
             }
             if (ok) umma_commit_elect(acc_done);
             umma_commit_elect(mma_done);
@@ -483,8 +591,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(mma_done, 0, drain);
         }
     } else if (warp >= kComputeWarp0) {
-        const int r = threadIdx.x - kComputeWarp0 * 32;
-        const uint32_t lane_off = static_cast<uint32_t>((warp - kComputeWarp0) * 32) << 16;
+        // ------------------------------------------------ element-wise: thread = query row r, 64 key columns
+        const int quad = warp & 3, half = (warp - kComputeWarp0) >> 2;
+        const int r = quad * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int i = qt * kTileM + r;
         const bool valid = i < p.N;
         const int lo = valid ? p.doc_start[i] : i;
@@ -493,55 +603,77 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float sl2 = p.scale_log2;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            const int c0 = (kt0 + j) * kTileN;
-            if (!mbar_wait(s_full, j & 1, wc)) { ok = false; break; }
+            const int c0 = (kt0 + j) * kTileN + half * 64;   // first key of this half
+            const uint32_t tS = tbase + ((j & 1) ? C::T_S2 : C::T_S) + lane_off + half * 64;
+            if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const bool need_mask = (c0 < lo) || (c0 + kTileN - 1 > i);
-            const bool any_mask = __any_sync(0xffffffffu, need_mask);
+            const bool any_mask = __any_sync(0xffffffffu, (c0 < lo) || (c0 + 63 > i));
+            // phase 1 (while dP(j) may still be computing): P = exp2(S * scale*log2(e)
+            // - LSE*log2(e)), kept as bf16 pairs
+            uint32_t pp[32];
+            {
+                uint32_t sr[64];
+                tmem_ld64(tS, sr);
+                tmem_ld_wait();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sr[64], dr[64];
-                tmem_ld64(tbase + C::T_S + lane_off + half * 64, sr);
+                for (int e = 0; e < 32; ++e) {
+                    float x0, x1;
+                    fma2_bcast(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, nl2);
+                    if (any_mask) {
+                        const int key = c0 + 2 * e;
+                        if (key < lo || key > i) x0 = -CUDART_INF_F;
+                        if (key + 1 < lo || key + 1 > i) x1 = -CUDART_INF_F;
+                    }
+                    float p0, p1;
+                    if ((e & 7) < kBwdEmuPairs) {
+                        ex2_poly2(p0, p1, x0, x1);
+                    } else {
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
+                    pp[e] = pack_bf16x2(p0, p1);
+                }
+            }
+            // phase 2: dS = P (dP - D) from the bf16 P, bf16 into S's columns
+            if (!mbar_wait(dp_full, j & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t dr[64];
                 tmem_ld64(tbase + C::T_DP + lane_off + half * 64, dr);
                 tmem_ld_wait();
                 uint32_t dd[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int c = half * 64 + 2 * e;
-                    float x0, x1;
-                    fma2_bcast(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, nl2);
-                    if (any_mask) {
-                        if (c0 + c < lo || c0 + c > i) x0 = -CUDART_INF_F;
-                        if (c0 + c + 1 < lo || c0 + c + 1 > i) x1 = -CUDART_INF_F;
-                    }
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    const uint32_t pe = pp[e];
                     float t0, t1, d0, d1;
                     sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), di, di);
-                    mul2(d0, d1, p0, p1, t0, t1);
+                    mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
                     dd[e] = pack_bf16x2(d0, d1);
                 }
-                tmem_st32(tbase + C::T_S + lane_off + half * 32, dd);   // dS (keys packed in pairs)
+                tmem_st32(tS, dd);   // dS (keys packed in pairs)
             }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(ds_full);
         }
+        // ---- epilogue: this half writes d columns [half * D/2, (half + 1) * D/2) of dQ
         if (ok && mbar_wait(acc_done, 0, wc)) {
             tc_fence_after();
-            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hl + h) * D;
+            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hl + h) * D + half * (D / 2);
+            const uint32_t tacc = tbase + C::T_ACC0 + lane_off + half * (D / 2);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t raw[32];
-                tmem_ld32(tbase + C::T_ACC0 + lane_off + c * 32, raw);
+                uint32_t raw[16];
+                tmem_ld16(tacc + c * 16, raw);
                 tmem_ld_wait();
-                uint32_t w[16];
+                uint32_t w[8];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
+                for (int e = 0; e < 8; ++e)
                     w[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * p.scale, __uint_as_float(raw[2 * e + 1]) * p.scale);
                 if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(row + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    uint4 *dst = reinterpret_cast<uint4 *>(row + c * 16);
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
         }

@@ -59,6 +59,28 @@ def test_fwd_scale_argument():
     assert_close("LSE", lse.double().cpu().numpy(), rl)
 
 
+def test_fwd_rising_and_jumping_scores():
+    """Scores that rise along the sequence (the running maximum of a row grows
+    by far more than 2^8 across its key tiles) and one key tile whose scores
+    jump by more than 128 in log2 units (its exponentials overflow against the old
+    offset): both force the kernel's slow path, which reloads S, takes the row
+    maximum and rescales O and the row sum."""
+    N, Hl, Hkvl, d = 1000, 2, 1, 128
+    lengths = [700, 300]
+    c = random_case(N, Hl, Hkvl, d, lengths, seed=11, device="cuda")
+    j = torch.arange(N, device="cuda", dtype=torch.float32)[:, None, None]
+    q = c["q"].float().abs()
+    k = 0.25 * c["k"].float() + 3.0 * j / N
+    k[640:672] += 12.0
+    c["q"] = q.to(torch.bfloat16)
+    c["k"] = k.to(torch.bfloat16)
+    o, lse = _run(c)
+    ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    assert np.isfinite(lse.double().cpu().numpy()).all()
+    assert_close("O", bf16_to_f64(o), ro)
+    assert_close("LSE", lse.double().cpu().numpy(), rl, rel=1e-5)
+
+
 def test_fwd_one_token_documents_return_v():
     N, Hl, Hkvl, d = 384, 4, 2, 128
     c = random_case(N, Hl, Hkvl, d, [1] * N, seed=1, device="cuda")
