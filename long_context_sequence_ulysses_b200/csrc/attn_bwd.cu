@@ -351,19 +351,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float *rl = sRow + (s * 2 + 0) * 128 + half * 64;   // -lse2 of this half's queries
             const float *rd = sRow + (s * 2 + 1) * 128 + half * 64;   // delta of this half's queries
             const bool any_mask = __any_sync(0xffffffffu, (q0 < j) || (q0 + 63 >= dend));
-            // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns
+            // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns.
+            // Two chunks of 32 columns; each chunk's per-query values are fetched
+            // from shared memory as float4 before waiting for the tensor-memory load.
             uint32_t pp[32];
-            {
-                uint32_t sr[64];
-                tmem_ld64(tbase + C::T_S + lane_off + half * 64, sr);
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+                uint32_t sr[32];
+                tmem_ld32(tbase + C::T_S + lane_off + half * 64 + sub * 32, sr);
+                float4 nl[8];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) nl[v] = *reinterpret_cast<const float4 *>(rl + sub * 32 + 4 * v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float2 nl = *reinterpret_cast<const float2 *>(rl + 2 * e);
+                for (int e = 0; e < 16; ++e) {
+                    const float4 &n4 = nl[e >> 1];
+                    const float a0 = (e & 1) ? n4.z : n4.x, a1 = (e & 1) ? n4.w : n4.y;
                     float x0, x1;
-                    fma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, nl.x, nl.y);
+                    fma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, a0, a1);
                     if (any_mask) {
-                        const int qi = q0 + 2 * e;
+                        const int qi = q0 + sub * 32 + 2 * e;
                         if (qi < j || qi >= dend) x0 = -CUDART_INF_F;
                         if (qi + 1 < j || qi + 1 >= dend) x1 = -CUDART_INF_F;
                     }
@@ -374,10 +381,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         p0 = ex2_approx(x0);
                         p1 = ex2_approx(x1);
                     }
-                    pp[e] = pack_bf16x2(p0, p1);
+                    pp[sub * 16 + e] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32(tbase + C::T_S + lane_off + half * 64, pp);   // P^T (queries packed in pairs)
             }
+            tmem_st32(tbase + C::T_S + lane_off + half * 64, pp);   // P^T (queries packed in pairs)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_ready);
@@ -385,18 +392,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!mbar_wait(dp_full, it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
-                uint32_t dr[64];
-                tmem_ld64(tbase + C::T_DP + lane_off + half * 64, dr);
-                tmem_ld_wait();
                 uint32_t dd[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float2 dl = *reinterpret_cast<const float2 *>(rd + 2 * e);
-                    const uint32_t pe = pp[e];
-                    float t0, t1, d0, d1;
-                    sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), dl.x, dl.y);
-                    mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
-                    dd[e] = pack_bf16x2(d0, d1);
+                for (int sub = 0; sub < 2; ++sub) {
+                    uint32_t dr[32];
+                    tmem_ld32(tbase + C::T_DP + lane_off + half * 64 + sub * 32, dr);
+                    float4 dl[8];
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) dl[v] = *reinterpret_cast<const float4 *>(rd + sub * 32 + 4 * v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float4 &d4 = dl[e >> 1];
+                        const float b0 = (e & 1) ? d4.z : d4.x, b1 = (e & 1) ? d4.w : d4.y;
+                        const uint32_t pe = pp[sub * 16 + e];
+                        float t0, t1, d0, d1;
+                        sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), b0, b1);
+                        mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
+                        dd[sub * 16 + e] = pack_bf16x2(d0, d1);
+                    }
                 }
                 tmem_st32(tbase + C::T_DP + lane_off + half * 64, dd);   // dS^T
             }
