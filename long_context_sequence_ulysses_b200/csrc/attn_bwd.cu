@@ -25,6 +25,10 @@
 //     and dP^T(i+1) run while P^T(i+1) is computed.
 //  3. dQ: one CTA per (query tile, head) loops over its key tiles:
 //       S = Q K^T, dP = dO V^T -> dS (bf16, into S's columns) -> dQ += dS K.
+//     S has two buffers (the second in the columns the dQ accumulator leaves
+//     free) and runs two key tiles ahead: P is formed while dP is computed,
+//     and dQ, the next dP and the S after next run while the element-wise
+//     step of the following tile proceeds.
 #include "ptx.cuh"
 #include "ulysses_internal.cuh"
 
