@@ -39,17 +39,19 @@ namespace uly {
 
 namespace {
 
-// Warps 0..3: producers and the MMA issuer; warps 4..11: the element-wise
+// Warps 0..3: producers and the MMA issuer; warps 4..19: the element-wise
 // step. Compute warp w handles the 32 TMEM lanes (rows) of quarter w % 4 and
-// half (w - 4) / 4 of the 128 columns: the special-function unit and the
-// latency of each phase are shared by two warps per SM sub-partition. Each half
-// writes its bf16 results to its own 32-column region (half 0: columns 0..31,
-// half 1: columns 64..95 of the tile's 128), so neither overwrites columns
-// the other still has to read; the TS MMAs take K steps 4..7 from +64.
-constexpr int kBwdThreads = 384;
+// part (w - 4) / 4 of the 128 columns (kPartCols each): four warps per SM
+// sub-partition hide each other's latency in the exponential and product
+// phases. Each part writes its bf16 results to the first half of its own
+// columns, so no part overwrites columns another still has to read; the TS
+// MMAs find K step kk (16 rows, 8 packed columns) at pcol(kk).
+// All exponentials go to the SFU here: moving part of them to the FMA-pipe
+// polynomial (as the forward does) measured slower in both kernels.
+constexpr int kParts = 4;
+constexpr int kPartCols = kTileN / kParts;
+constexpr int kBwdThreads = 128 + kParts * 128;
 constexpr int kComputeWarp0 = 4;
-// Column pairs (out of every 8) whose exponentials run on the FMA pipe.
-constexpr int kBwdEmuPairs = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -154,8 +156,13 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
 }
 
 // Column of the bf16 operand packed in tensor memory for K step kk (16 rows
-// of the 128, two per column): half 0 wrote columns 0..31, half 1 64..95.
-__device__ __forceinline__ uint32_t pcol(int kk) { return static_cast<uint32_t>(kk * 8 + (kk >= 4 ? 32 : 0)); }
+// of the 128, two per column): part q wrote the 16-row steps of its columns
+// into columns q * kPartCols + 0 .. kPartCols / 2 - 1.
+__device__ __forceinline__ uint32_t pcol(int kk)
+{
+    constexpr int steps = kPartCols / 16;   // K steps per part
+    return static_cast<uint32_t>((kk / steps) * kPartCols + (kk % steps) * 8);
+}
 
 // K-major SS descriptors for a 16-element K step kk of a 128-row tile.
 template <int D>
@@ -204,9 +211,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *qdo_full = bars + 1;            // [NST]
     uint64_t *qdo_empty = qdo_full + C::NST;  // [NST]
     uint64_t *s_full = qdo_empty + C::NST;   // S^T(i) computed
-    uint64_t *ds_full = s_full + 1;           // dS^T(i) stored (256 arrivals)
+    uint64_t *ds_full = s_full + 1;           // dS^T(i) stored (all compute threads)
     uint64_t *dp_full = ds_full + 1;          // dP^T(i) computed
-    uint64_t *p_ready = dp_full + 1;          // P^T(i) stored (256 arrivals)
+    uint64_t *p_ready = dp_full + 1;          // P^T(i) stored (all compute threads)
     uint64_t *acc_done = p_ready + 1;
     uint64_t *mma_done = acc_done + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
@@ -227,9 +234,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&qdo_empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(ds_full, 256);
+        mbar_init(ds_full, kParts * 128);
         mbar_init(dp_full, 1);
-        mbar_init(p_ready, 256);
+        mbar_init(p_ready, kParts * 128);
         mbar_init(acc_done, 1);
         mbar_init(mma_done, 1);
         fence_mbar_init();
@@ -329,8 +336,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(mma_done, 0, drain);
         }
     } else if (warp >= kComputeWarp0) {
-        // ------------------------------------------------ element-wise: thread = key row r, 64 query columns
-        const int quad = warp & 3, half = (warp - kComputeWarp0) >> 2;
+        // ------------------------------------------------ element-wise: thread = key row r, kPartCols query columns
+        const int quad = warp & 3, part = (warp - kComputeWarp0) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int j = t * kTileN + r;
@@ -345,50 +352,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dend = hi;
         }
         const float sl2 = p.scale_log2;
+        const uint32_t col = static_cast<uint32_t>(part * kPartCols);   // this part's columns in S^T / dP^T
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int s = it % C::NST, u = it / C::NST;
-            const int q0 = (qt0 + it % n_q) * kTileM + half * 64;   // first query of this half
+            const int q0 = (qt0 + it % n_q) * kTileM + part * kPartCols;   // first query of this part
             if (!mbar_wait(s_full, it & 1, wc)) { ok = false; break; }
             if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const float *rl = sRow + (s * 2 + 0) * 128 + half * 64;   // -lse2 of this half's queries
-            const float *rd = sRow + (s * 2 + 1) * 128 + half * 64;   // delta of this half's queries
-            const bool any_mask = __any_sync(0xffffffffu, (q0 < j) || (q0 + 63 >= dend));
-            // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns.
-            // Two chunks of 32 columns; each chunk's per-query values are fetched
-            // from shared memory as float4 before waiting for the tensor-memory load.
-            uint32_t pp[32];
+            const float *rl = sRow + (s * 2 + 0) * 128 + part * kPartCols;   // -lse2 of this part's queries
+            const float *rd = sRow + (s * 2 + 1) * 128 + part * kPartCols;   // delta of this part's queries
+            const bool any_mask = __any_sync(0xffffffffu, (q0 < j) || (q0 + kPartCols - 1 >= dend));
+            // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns;
+            // the per-query values are fetched as float4 before waiting for the tensor-memory load
+            uint32_t pp[kPartCols / 2];
+            {
+                uint32_t sr[kPartCols];
+                tmem_ld32(tbase + C::T_S + lane_off + col, sr);
+                float4 nl[kPartCols / 4];
 #pragma unroll
-            for (int sub = 0; sub < 2; ++sub) {
-                uint32_t sr[32];
-                tmem_ld32(tbase + C::T_S + lane_off + half * 64 + sub * 32, sr);
-                float4 nl[8];
-#pragma unroll
-                for (int v = 0; v < 8; ++v) nl[v] = *reinterpret_cast<const float4 *>(rl + sub * 32 + 4 * v);
+                for (int v = 0; v < kPartCols / 4; ++v) nl[v] = *reinterpret_cast<const float4 *>(rl + 4 * v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
+                for (int e = 0; e < kPartCols / 2; ++e) {
                     const float4 &n4 = nl[e >> 1];
                     const float a0 = (e & 1) ? n4.z : n4.x, a1 = (e & 1) ? n4.w : n4.y;
                     float x0, x1;
                     fma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, a0, a1);
                     if (any_mask) {
-                        const int qi = q0 + sub * 32 + 2 * e;
+                        const int qi = q0 + 2 * e;
                         if (qi < j || qi >= dend) x0 = -CUDART_INF_F;
                         if (qi + 1 < j || qi + 1 >= dend) x1 = -CUDART_INF_F;
                     }
-                    float p0, p1;
-                    if ((e & 7) < kBwdEmuPairs) {
-                        ex2_poly2(p0, p1, x0, x1);
-                    } else {
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
-                    }
-                    pp[sub * 16 + e] = pack_bf16x2(p0, p1);
+                    pp[e] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
                 }
             }
-            tmem_st32(tbase + C::T_S + lane_off + half * 64, pp);   // P^T (queries packed in pairs)
+            tmem_st16(tbase + C::T_S + lane_off + col, pp);   // P^T (queries packed in pairs)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_ready);
@@ -396,45 +395,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!mbar_wait(dp_full, it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
-                uint32_t dd[32];
+                uint32_t dr[kPartCols];
+                tmem_ld32(tbase + C::T_DP + lane_off + col, dr);
+                float4 dl[kPartCols / 4];
 #pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    uint32_t dr[32];
-                    tmem_ld32(tbase + C::T_DP + lane_off + half * 64 + sub * 32, dr);
-                    float4 dl[8];
+                for (int v = 0; v < kPartCols / 4; ++v) dl[v] = *reinterpret_cast<const float4 *>(rd + 4 * v);
+                tmem_ld_wait();
+                uint32_t dd[kPartCols / 2];
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) dl[v] = *reinterpret_cast<const float4 *>(rd + sub * 32 + 4 * v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float4 &d4 = dl[e >> 1];
-                        const float b0 = (e & 1) ? d4.z : d4.x, b1 = (e & 1) ? d4.w : d4.y;
-                        const uint32_t pe = pp[sub * 16 + e];
-                        float t0, t1, d0, d1;
-                        sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), b0, b1);
-                        mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
-                        dd[sub * 16 + e] = pack_bf16x2(d0, d1);
-                    }
+                for (int e = 0; e < kPartCols / 2; ++e) {
+                    const float4 &d4 = dl[e >> 1];
+                    const float b0 = (e & 1) ? d4.z : d4.x, b1 = (e & 1) ? d4.w : d4.y;
+                    const uint32_t pe = pp[e];
+                    float t0, t1, d0, d1;
+                    sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), b0, b1);
+                    mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
+                    dd[e] = pack_bf16x2(d0, d1);
                 }
-                tmem_st32(tbase + C::T_DP + lane_off + half * 64, dd);   // dS^T
+                tmem_st16(tbase + C::T_DP + lane_off + col, dd);   // dS^T
             }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(ds_full);
         }
-        // ---- epilogue: this half writes d columns [half * D/2, (half + 1) * D/2) of dV and dK
-        if (ok && mbar_wait(acc_done, 0, wc)) {
+        // ---- epilogue: part p writes d columns [p * E, (p + 1) * E) of dV and dK, E = max(16, D / kParts)
+        constexpr int E = (D / kParts) >= 16 ? D / kParts : 16;
+        if (ok && part * E < D && mbar_wait(acc_done, 0, wc)) {
             tc_fence_after();
             const bool valid = j < p.N;
-            __nv_bfloat16 *dv_row = p.dv + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + half * (D / 2);
-            __nv_bfloat16 *dk_row = p.dk + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + half * (D / 2);
+            __nv_bfloat16 *dv_row = p.dv + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + part * E;
+            __nv_bfloat16 *dk_row = p.dk + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + part * E;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const float mul = which == 0 ? 1.f : p.scale;
                 __nv_bfloat16 *row = which == 0 ? dv_row : dk_row;
-                const uint32_t tacc = tbase + (which == 0 ? C::T_ACC0 : C::T_ACC1) + lane_off + half * (D / 2);
+                const uint32_t tacc = tbase + (which == 0 ? C::T_ACC0 : C::T_ACC1) + lane_off + part * E;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < E / 16; ++c) {
                     uint32_t raw[16];
                     tmem_ld16(tacc + c * 16, raw);
                     tmem_ld_wait();
@@ -480,7 +477,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *v_empty = v_full + C::QVST;    // [QVST] dP(j) has read V_j
     uint64_t *s_full = v_empty + C::QVST;    // [2] S(j) computed into buffer j % 2
     uint64_t *dp_full = s_full + 2;          // dP(j) computed
-    uint64_t *ds_full = dp_full + 1;         // dS(j) stored (256 arrivals)
+    uint64_t *ds_full = dp_full + 1;         // dS(j) stored (all compute threads)
     uint64_t *acc_done = ds_full + 1;
     uint64_t *mma_done = acc_done + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
@@ -506,7 +503,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
         mbar_init(dp_full, 1);
-        mbar_init(ds_full, 256);
+        mbar_init(ds_full, kParts * 128);
         mbar_init(acc_done, 1);
         mbar_init(mma_done, 1);
         fence_mbar_init();
@@ -609,8 +606,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(mma_done, 0, drain);
         }
     } else if (warp >= kComputeWarp0) {
-        // ------------------------------------------------ element-wise: thread = query row r, 64 key columns
-        const int quad = warp & 3, half = (warp - kComputeWarp0) >> 2;
+        // ------------------------------------------------ element-wise: thread = query row r, kPartCols key columns
+        const int quad = warp & 3, part = (warp - kComputeWarp0) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int i = qt * kTileM + r;
@@ -619,22 +616,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float nl2 = p.lse2[static_cast<int64_t>(h) * p.Npad + i];   // -LSE * log2(e)
         const float di = p.delta[static_cast<int64_t>(h) * p.Npad + i];
         const float sl2 = p.scale_log2;
+        const uint32_t col = static_cast<uint32_t>(part * kPartCols);
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            const int c0 = (kt0 + j) * kTileN + half * 64;   // first key of this half
-            const uint32_t tS = tbase + ((j & 1) ? C::T_S2 : C::T_S) + lane_off + half * 64;
+            const int c0 = (kt0 + j) * kTileN + part * kPartCols;   // first key of this part
+            const uint32_t tS = tbase + ((j & 1) ? C::T_S2 : C::T_S) + lane_off + col;
             if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const bool any_mask = __any_sync(0xffffffffu, (c0 < lo) || (c0 + 63 > i));
+            const bool any_mask = __any_sync(0xffffffffu, (c0 < lo) || (c0 + kPartCols - 1 > i));
             // phase 1 (while dP(j) may still be computing): P = exp2(S * scale*log2(e)
             // - LSE*log2(e)), kept as bf16 pairs
-            uint32_t pp[32];
+            uint32_t pp[kPartCols / 2];
             {
-                uint32_t sr[64];
-                tmem_ld64(tS, sr);
+                uint32_t sr[kPartCols];
+                tmem_ld32(tS, sr);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
+                for (int e = 0; e < kPartCols / 2; ++e) {
                     float x0, x1;
                     fma2_bcast(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, nl2);
                     if (any_mask) {
@@ -642,45 +640,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         if (key < lo || key > i) x0 = -CUDART_INF_F;
                         if (key + 1 < lo || key + 1 > i) x1 = -CUDART_INF_F;
                     }
-                    float p0, p1;
-                    if ((e & 7) < kBwdEmuPairs) {
-                        ex2_poly2(p0, p1, x0, x1);
-                    } else {
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
-                    }
-                    pp[e] = pack_bf16x2(p0, p1);
+                    pp[e] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
                 }
             }
             // phase 2: dS = P (dP - D) from the bf16 P, bf16 into S's columns
             if (!mbar_wait(dp_full, j & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
-                uint32_t dr[64];
-                tmem_ld64(tbase + C::T_DP + lane_off + half * 64, dr);
+                uint32_t dr[kPartCols];
+                tmem_ld32(tbase + C::T_DP + lane_off + col, dr);
                 tmem_ld_wait();
-                uint32_t dd[32];
+                uint32_t dd[kPartCols / 2];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
+                for (int e = 0; e < kPartCols / 2; ++e) {
                     const uint32_t pe = pp[e];
                     float t0, t1, d0, d1;
                     sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), di, di);
                     mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
                     dd[e] = pack_bf16x2(d0, d1);
                 }
-                tmem_st32(tS, dd);   // dS (keys packed in pairs)
+                tmem_st16(tS, dd);   // dS (keys packed in pairs)
             }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(ds_full);
         }
-        // ---- epilogue: this half writes d columns [half * D/2, (half + 1) * D/2) of dQ
-        if (ok && mbar_wait(acc_done, 0, wc)) {
+        // ---- epilogue: part p writes d columns [p * E, (p + 1) * E) of dQ, E = max(16, D / kParts)
+        constexpr int E = (D / kParts) >= 16 ? D / kParts : 16;
+        if (ok && part * E < D && mbar_wait(acc_done, 0, wc)) {
             tc_fence_after();
-            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hl + h) * D + half * (D / 2);
-            const uint32_t tacc = tbase + C::T_ACC0 + lane_off + half * (D / 2);
+            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hl + h) * D + part * E;
+            const uint32_t tacc = tbase + C::T_ACC0 + lane_off + part * E;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < E / 16; ++c) {
                 uint32_t raw[16];
                 tmem_ld16(tacc + c * 16, raw);
                 tmem_ld_wait();
