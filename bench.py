@@ -221,6 +221,53 @@ def build_single(U, w, inp, dev, timed):
     return step, launches, ws
 
 
+def build_fused(U, w, inp, dev):
+    """One GPU, fused exchanges: every emulated rank's attention reads its head
+    slice straight from the sequence-sharded Q/K/V (and dO) and writes O (and
+    dQ/dK/dV) straight back into that layout, so no relayout runs.
+    Returns (step, our kernel launches per step, workspace)."""
+    P, N, d, Hl, Hkvl = w.P, w.N, w.d, w.Hl, w.Hkvl
+    pos = inp["position_ids"]
+    q_seq, k_seq, v_seq, do_seq = inp["q"], inp["k"], inp["v"], inp.get("do")
+    o_seq = torch.empty_like(q_seq)
+    lse_all = torch.empty((P * Hl, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, w.backward), dtype=torch.uint8, device=dev)
+    if w.backward:
+        dq_seq, dk_seq, dv_seq = torch.empty_like(q_seq), torch.empty_like(k_seq), torch.empty_like(v_seq)
+
+    def step():
+        for r in range(P):
+            U.attn_fwd_fused(q_seq, k_seq, v_seq, pos, P, r, out=o_seq, lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws)
+        if w.backward:
+            for r in range(P):
+                U.attn_bwd_fused(q_seq, k_seq, v_seq, o_seq, do_seq, lse_all[r * Hl:(r + 1) * Hl], pos, P, r,
+                                 dq=dq_seq, dk=dk_seq, dv=dv_seq, ws=ws)
+
+    return step, 4 * P + (BWD_LAUNCHES * P if w.backward else 0), ws
+
+
+def time_fused(U, w, inp, dev, steps, total_flop):
+    """The step with the exchanges fused into the attention (see build_fused)."""
+    step, launches, ws = build_fused(U, w, inp, dev)
+    stream = torch.cuda.current_stream(dev)
+    step()
+    torch.cuda.synchronize()
+    U.sync_status(ws)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    U.sync_status(ws)
+    ms = t0.elapsed_time(t1) / steps
+    return {"ms_per_step": round(ms, 4), "value": round(total_flop / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "gpu_launches": launches * steps,
+            "step": "attn_fwd_fused per rank" + ("; attn_bwd_fused per rank" if w.backward else "")
+                    + ": sequence-sharded Q/K/V in, O out, no relayout"}
+
+
 def build_multi(U, w, inp, dev, timed, G, rank):
     """G GPUs: Ulysses with P = G real ranks. Each GPU holds tokens
     [rank*N/G, (rank+1)*N/G); the pack before and the unpack after each NCCL
@@ -390,6 +437,8 @@ def run_gpu(args):
                            "frac": round(rb / peaks["hbm_gbs"], 4), "frac_of_spec_8000": round(rb / SPEC_HBM_GBS, 4)}
     if exch_sum:
         out["exchange_ms_per_step"] = round(exch_sum / args.steps, 4)
+    if world == 1 and args.fused:
+        out["fused_step"] = time_fused(U, w, inp, dev, args.steps, total_flop)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, inp, args)
     if dist is not None:
@@ -553,6 +602,8 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fused", dest="fused", action="store_false",
+                    help="skip the extra timing of the step with the exchanges fused into the attention")
     ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     args = ap.parse_args()

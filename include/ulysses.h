@@ -139,6 +139,26 @@ int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o,
                      void *dq, void *dk, void *dv, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Fused form of the backward, as ulysses_attn_fwd_fused is of the forward:
+ * rank `rank`'s head slice is read from the sequence-sharded buffers and its
+ * gradients are written straight into the sequence-sharded layout, so none
+ * of the backward's exchanges (dout in; dq, dk, dv out) is materialised.
+ *
+ *   q_seq, o_seq, dout_seq [N][H][d]; k_seq, v_seq [N][Hkv][d]
+ *         (= [P][N/P][heads][d]); lse [H/P][N] for this rank's heads.
+ *   dq_seq [N][H][d], dk_seq / dv_seq [N][Hkv][d]: only this rank's heads
+ *         ([rank*H/P, (rank+1)*H/P) and [rank*Hkv/P, (rank+1)*Hkv/P)) are
+ *         written, so the calls of all ranks together fill them.
+ * Same checks as ulysses_attn_fwd_fused; the workspace is the backward one for
+ * (N, H/P, Hkv/P, d).
+ */
+int ulysses_attn_bwd_fused(const void *q_seq, const void *k_seq, const void *v_seq,
+                           const void *o_seq, const void *dout_seq, const float *lse,
+                           const int32_t *position_ids, int64_t N, int P, int H, int Hkv,
+                           int d, int rank, float scale, void *dq_seq, void *dk_seq, void *dv_seq,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/*
  * No counterpart in the pages: ulysses_attn_fwd for callers that cannot
  * allocate device memory, such as a plugin inside a host framework that owns
  * all device memory through its own pool and hands over only input and output

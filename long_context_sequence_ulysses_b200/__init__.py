@@ -25,7 +25,8 @@ import torch
 
 __all__ = [
     "UlyssesError", "library_path", "seq_to_head", "head_to_seq", "workspace_bytes", "attn_fwd",
-    "attn_fwd_fused", "attn_bwd", "sync_status", "set_wait_limit_ns", "set_debug_flags", "version",
+    "attn_fwd_fused", "attn_bwd", "attn_bwd_fused", "sync_status", "set_wait_limit_ns", "set_debug_flags",
+    "version",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -61,13 +62,15 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_attn_fwd.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, SZ, P]
     lib.ulysses_attn_fwd_fused.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, F32, P, P, P, SZ, P]
     lib.ulysses_attn_bwd.argtypes = [P, P, P, P, P, P, P, I64, I32, I32, I32, F32, P, P, P, P, SZ, P]
+    lib.ulysses_attn_bwd_fused.argtypes = [P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, F32, P, P, P, P, SZ,
+                                           P]
     lib.ulysses_sync_status.argtypes = [P, P]
     lib.ulysses_set_wait_limit_ns.argtypes = [I64]
     lib.ulysses_set_wait_limit_ns.restype = None
     lib.ulysses_set_debug_flags.argtypes = [ctypes.c_uint32]
     lib.ulysses_set_debug_flags.restype = None
     for name in ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_fwd_fused",
-                 "ulysses_attn_bwd", "ulysses_sync_status"):
+                 "ulysses_attn_bwd", "ulysses_attn_bwd_fused", "ulysses_sync_status"):
         getattr(lib, name).restype = I32
     return lib
 
@@ -249,3 +252,31 @@ def set_debug_flags(flags: int) -> None:
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def attn_bwd_fused(q_seq: torch.Tensor, k_seq: torch.Tensor, v_seq: torch.Tensor, o_seq: torch.Tensor,
+                   dout_seq: torch.Tensor, lse: torch.Tensor, position_ids: torch.Tensor, P: int, rank: int,
+                   scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
+                   dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                   ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients of rank ``rank``'s heads read straight from the sequence-sharded
+    buffers (q/o/dout [N][H][d], k/v [N][Hkv][d]) and written into dq [N][H][d],
+    dk / dv [N][Hkv][d] (only this rank's heads); lse is [H/P][N]."""
+    for name, t in (("q_seq", q_seq), ("k_seq", k_seq), ("v_seq", v_seq), ("o_seq", o_seq), ("dout_seq", dout_seq)):
+        _bf16_cuda(name, t, 3)
+    N, H, d = q_seq.shape
+    Hkv = k_seq.shape[1]
+    Hl, Hkvl = H // P, Hkv // P
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (Hl, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [H/P][N] tensor")
+    pos = _pos32(position_ids, N)
+    dq = torch.empty_like(q_seq) if dq is None else dq
+    dk = torch.empty_like(k_seq) if dk is None else dk
+    dv = torch.empty_like(v_seq) if dv is None else dv
+    nbytes = workspace_bytes(N, max(Hl, 1), max(Hkvl, 1), d, True)
+    ws = _workspace(ws, nbytes, q_seq.device)
+    sc = 0.0 if scale is None else float(scale)
+    _check(_lib.ulysses_attn_bwd_fused(_ptr(q_seq), _ptr(k_seq), _ptr(v_seq), _ptr(o_seq), _ptr(dout_seq), _ptr(lse),
+                                       _ptr(pos), N, P, H, Hkv, d, rank, sc, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                       ws.numel(), _stream(q_seq)))
+    return dq, dk, dv

@@ -230,16 +230,14 @@ int ulysses_attn_fwd_fused(const void *q_seq, const void *k_seq, const void *v_s
                            stream, H, Hkv, rank * Hl, rank * Hkvl);
 }
 
-int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
-                     const int32_t *position_ids, int64_t N, int Hl, int Hkvl, int d, float scale, void *dq, void *dk,
-                     void *dv, void *ws, size_t ws_bytes, void *stream)
+// Shared by the slice and the fused (sequence-layout) backward entry points.
+static int attn_bwd_common(const char *name, const void *q, const void *k, const void *v, const void *o,
+                           const void *dout, const float *lse, const int32_t *position_ids, int64_t N, int Hl,
+                           int Hkvl, int d, float scale, void *dq, void *dk, void *dv, void *ws, size_t ws_bytes,
+                           void *stream, int Hq_total, int Hkv_total, int q_head0, int kv_head0)
 {
-    const char *name = "ulysses_attn_bwd";
-    g_err[0] = 0;
-    int rc = check_attn_shapes(name, N, Hl, Hkvl, d);
-    if (rc) return rc;
     WsLayout L = ws_layout(N, Hl, true);
-    rc = check_ws(name, ws, ws_bytes, L);
+    int rc = check_ws(name, ws, ws_bytes, L);
     if (rc) return rc;
     if (N == 0) return ULYSSES_OK;
     if (!q || !k || !v || !o || !dout || !lse || !position_ids || !dq || !dk || !dv)
@@ -256,6 +254,8 @@ int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o,
     a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
     a.dq = dq; a.dk = dk; a.dv = dv;
     a.N = N; a.Hl = Hl; a.Hkvl = Hkvl; a.d = d;
+    a.Hq_total = Hq_total; a.Hkv_total = Hkv_total;
+    a.q_head0 = q_head0; a.kv_head0 = kv_head0;
     a.scale = scale;
     a.ws = static_cast<char *>(ws);
     a.L = L;
@@ -264,6 +264,38 @@ int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o,
     if (e == cudaErrorNotSupported) return fail(ULYSSES_ERR_UNSUPPORTED, "%s: not built", name);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return ULYSSES_OK;
+}
+
+int ulysses_attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+                     const int32_t *position_ids, int64_t N, int Hl, int Hkvl, int d, float scale, void *dq, void *dk,
+                     void *dv, void *ws, size_t ws_bytes, void *stream)
+{
+    const char *name = "ulysses_attn_bwd";
+    g_err[0] = 0;
+    int rc = check_attn_shapes(name, N, Hl, Hkvl, d);
+    if (rc) return rc;
+    return attn_bwd_common(name, q, k, v, o, dout, lse, position_ids, N, Hl, Hkvl, d, scale, dq, dk, dv, ws, ws_bytes,
+                           stream, Hl, Hkvl, 0, 0);
+}
+
+int ulysses_attn_bwd_fused(const void *q_seq, const void *k_seq, const void *v_seq, const void *o_seq,
+                           const void *dout_seq, const float *lse, const int32_t *position_ids, int64_t N, int P,
+                           int H, int Hkv, int d, int rank, float scale, void *dq_seq, void *dk_seq, void *dv_seq,
+                           void *ws, size_t ws_bytes, void *stream)
+{
+    const char *name = "ulysses_attn_bwd_fused";
+    g_err[0] = 0;
+    if (P < 1) return fail(ULYSSES_ERR_INVALID, "%s: P=%d < 1", name, P);
+    if (H < 1 || Hkv < 1) return fail(ULYSSES_ERR_INVALID, "%s: head counts must be >= 1", name);
+    if (H % P || Hkv % P)
+        return fail(ULYSSES_ERR_INVALID, "%s: H=%d and Hkv=%d must be divisible by P=%d", name, H, Hkv, P);
+    if (N % P) return fail(ULYSSES_ERR_INVALID, "%s: N=%lld not divisible by P=%d", name, (long long)N, P);
+    if (rank < 0 || rank >= P) return fail(ULYSSES_ERR_INVALID, "%s: rank=%d outside [0,%d)", name, rank, P);
+    const int Hl = H / P, Hkvl = Hkv / P;
+    int rc = check_attn_shapes(name, N, Hl, Hkvl, d);
+    if (rc) return rc;
+    return attn_bwd_common(name, q_seq, k_seq, v_seq, o_seq, dout_seq, lse, position_ids, N, Hl, Hkvl, d, scale,
+                           dq_seq, dk_seq, dv_seq, ws, ws_bytes, stream, H, Hkv, rank * Hl, rank * Hkvl);
 }
 
 int ulysses_sync_status(void *ws, void *stream)

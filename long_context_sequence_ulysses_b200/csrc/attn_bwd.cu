@@ -65,6 +65,8 @@ struct BwdParams {
     const float *lse2;    // [Hl][Npad]: -LSE * log2(e) (-inf on padding rows)
     __nv_bfloat16 *dq, *dk, *dv;
     int N, Npad, T, Hl, Hkvl;
+    int Hq_total, Hkv_total;   // heads per token row of the q / kv-side buffers
+    int q_head0, kv_head0;     // this slice's first head in those rows
     float scale_log2, scale;
     uint32_t *status;
     uint64_t wait_limit_ns;
@@ -126,7 +128,8 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
                                                       const __nv_bfloat16 *__restrict__ dout,
                                                       const float *__restrict__ lse, float *__restrict__ delta,
-                                                      float *__restrict__ lse2, int N, int Npad, int Hl)
+                                                      float *__restrict__ lse2, int N, int Npad, int Hl,
+                                                      int Hq_total, int q_head0)
 {
     const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -135,8 +138,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
     const int i = static_cast<int>(w % Npad);
     float acc = 0.f;
     if (i < N) {
-        const uint4 *po = reinterpret_cast<const uint4 *>(o + (static_cast<int64_t>(i) * Hl + h) * D);
-        const uint4 *pd = reinterpret_cast<const uint4 *>(dout + (static_cast<int64_t>(i) * Hl + h) * D);
+        const int64_t off = (static_cast<int64_t>(i) * Hq_total + q_head0 + h) * D;
+        const uint4 *po = reinterpret_cast<const uint4 *>(o + off);
+        const uint4 *pd = reinterpret_cast<const uint4 *>(dout + off);
         for (int v = lane; v < D / 8; v += 32) acc += dot8_bf16(po[v], pd[v]);
     }
 #pragma unroll
@@ -255,8 +259,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ------------------------------------------------ producer
         if (lane == 0) {
             mbar_arrive_expect_tx(kv_full, 2 * C::TILE_BYTES);
-            tma_tile<D>(&tmK, sK, kv_full, kvh, t * kTileN);
-            tma_tile<D>(&tmV, sV, kv_full, kvh, t * kTileN);
+            tma_tile<D>(&tmK, sK, kv_full, p.kv_head0 + kvh, t * kTileN);
+            tma_tile<D>(&tmV, sV, kv_full, p.kv_head0 + kvh, t * kTileN);
             int last_use[C::NST];
 #pragma unroll
             for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
@@ -266,8 +270,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int qt = qt0 + it % n_q;
                 if (u > 0 && !mbar_wait(&qdo_empty[s], (u - 1) & 1, wc)) break;
                 mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES + 2 * 512);
-                tma_tile<D>(&tmQ, sQ + s * C::TILE_BYTES, &qdo_full[s], h, qt * kTileM);
-                tma_tile<D>(&tmDO, sDO + s * C::TILE_BYTES, &qdo_full[s], h, qt * kTileM);
+                tma_tile<D>(&tmQ, sQ + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
+                tma_tile<D>(&tmDO, sDO + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
                 const int64_t roff = static_cast<int64_t>(h) * p.Npad + static_cast<int64_t>(qt) * kTileM;
                 bulk_load(sRow + (s * 2 + 0) * 128, p.lse2 + roff, 512, &qdo_full[s]);
                 bulk_load(sRow + (s * 2 + 1) * 128, p.delta + roff, 512, &qdo_full[s]);
@@ -423,8 +427,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (ok && part * E < D && mbar_wait(acc_done, 0, wc)) {
             tc_fence_after();
             const bool valid = j < p.N;
-            __nv_bfloat16 *dv_row = p.dv + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + part * E;
-            __nv_bfloat16 *dk_row = p.dk + (static_cast<int64_t>(j) * p.Hkvl + kvh) * D + part * E;
+            const int64_t kv_off = (static_cast<int64_t>(j) * p.Hkv_total + p.kv_head0 + kvh) * D + part * E;
+            __nv_bfloat16 *dv_row = p.dv + kv_off;
+            __nv_bfloat16 *dk_row = p.dk + kv_off;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const float mul = which == 0 ? 1.f : p.scale;
@@ -522,8 +527,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ------------------------------------------------ Q, dO and K producer
         if (lane == 0) {
             mbar_arrive_expect_tx(qdo_full, 2 * C::TILE_BYTES);
-            tma_tile<D>(&tmQ, sQ, qdo_full, h, qt * kTileM);
-            tma_tile<D>(&tmDO, sDO, qdo_full, h, qt * kTileM);
+            tma_tile<D>(&tmQ, sQ, qdo_full, p.q_head0 + h, qt * kTileM);
+            tma_tile<D>(&tmDO, sDO, qdo_full, p.q_head0 + h, qt * kTileM);
             int last_use[C::QKST];
 #pragma unroll
             for (int s = 0; s < C::QKST; ++s) last_use[s] = -1;
@@ -531,7 +536,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int s = j % C::QKST, u = j / C::QKST;
                 if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) break;
                 mbar_arrive_expect_tx(&k_full[s], C::TILE_BYTES);
-                tma_tile<D>(&tmK, sK + s * C::TILE_BYTES, &k_full[s], kvh, (kt0 + j) * kTileN);
+                tma_tile<D>(&tmK, sK + s * C::TILE_BYTES, &k_full[s], p.kv_head0 + kvh, (kt0 + j) * kTileN);
                 last_use[s] = u;
             }
             WaitCtx drain{p.wait_limit_ns, p.status, false};
@@ -549,7 +554,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int s = j % C::QVST, u = j / C::QVST;
                 if (u > 0 && !mbar_wait(&v_empty[s], (u - 1) & 1, wc)) break;
                 mbar_arrive_expect_tx(&v_full[s], C::TILE_BYTES);
-                tma_tile<D>(&tmV, sV + s * C::TILE_BYTES, &v_full[s], kvh, (kt0 + j) * kTileN);
+                tma_tile<D>(&tmV, sV + s * C::TILE_BYTES, &v_full[s], p.kv_head0 + kvh, (kt0 + j) * kTileN);
                 last_use[s] = u;
             }
             WaitCtx drain{p.wait_limit_ns, p.status, false};
@@ -669,7 +674,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         constexpr int E = (D / kParts) >= 16 ? D / kParts : 16;
         if (ok && part * E < D && mbar_wait(acc_done, 0, wc)) {
             tc_fence_after();
-            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hl + h) * D + part * E;
+            __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hq_total + p.q_head0 + h) * D + part * E;
             const uint32_t tacc = tbase + C::T_ACC0 + lane_off + part * E;
 #pragma unroll
             for (int c = 0; c < E / 16; ++c) {
@@ -716,11 +721,11 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     const int T = static_cast<int>(ceil_div(a.N, kTileM));
     const int Npad = T * kTileM;
     alignas(64) CUtensorMap tq, tk, tv, tdo;
-    const int64_t qs = int64_t(a.Hl) * D * 2, ks = int64_t(a.Hkvl) * D * 2;
-    if (!encode_tmap_3d(&tq, a.q, D, a.Hl, a.N, int64_t(D) * 2, qs, C::AW, kTileM, C::SW) ||
-        !encode_tmap_3d(&tdo, a.dout, D, a.Hl, a.N, int64_t(D) * 2, qs, C::AW, kTileM, C::SW) ||
-        !encode_tmap_3d(&tk, a.k, D, a.Hkvl, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW) ||
-        !encode_tmap_3d(&tv, a.v, D, a.Hkvl, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW))
+    const int64_t qs = int64_t(a.Hq_total) * D * 2, ks = int64_t(a.Hkv_total) * D * 2;
+    if (!encode_tmap_3d(&tq, a.q, D, a.Hq_total, a.N, int64_t(D) * 2, qs, C::AW, kTileM, C::SW) ||
+        !encode_tmap_3d(&tdo, a.dout, D, a.Hq_total, a.N, int64_t(D) * 2, qs, C::AW, kTileM, C::SW) ||
+        !encode_tmap_3d(&tk, a.k, D, a.Hkv_total, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW) ||
+        !encode_tmap_3d(&tv, a.v, D, a.Hkv_total, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW))
         return cudaErrorInvalidValue;
     BwdParams p;
     p.doc_start = reinterpret_cast<const int32_t *>(a.ws + a.L.doc_start);
@@ -740,6 +745,10 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     p.T = T;
     p.Hl = a.Hl;
     p.Hkvl = a.Hkvl;
+    p.Hq_total = a.Hq_total;
+    p.Hkv_total = a.Hkv_total;
+    p.q_head0 = a.q_head0;
+    p.kv_head0 = a.kv_head0;
     p.scale = a.scale;
     p.scale_log2 = a.scale * kLog2e;
     p.status = reinterpret_cast<uint32_t *>(a.ws + a.L.status);
@@ -748,7 +757,7 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     const int64_t prep_threads = int64_t(a.Hl) * Npad * 32;
     bwd_prep_kernel<D><<<static_cast<unsigned>(ceil_div(prep_threads, 256)), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, delta, lse2,
-        p.N, Npad, a.Hl);
+        p.N, Npad, a.Hl, a.Hq_total, a.q_head0);
     static bool kv_attr[64] = {}, q_attr[64] = {};
     cudaError_t e = set_smem(attn_bwd_dkdv_kernel<D>, C::KV_SMEM, kv_attr);
     if (e != cudaSuccess) return e;

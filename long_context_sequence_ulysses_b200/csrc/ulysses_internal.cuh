@@ -89,11 +89,13 @@ cudaError_t launch_attn_fwd(const FwdLaunch &a, cudaStream_t stream);
 
 // Backward attention launch description (no fused layout: slice buffers).
 struct BwdLaunch {
-    const void *q, *k, *v, *o, *dout;
+    const void *q, *k, *v, *o, *dout;   // [N][Hq_total][d] (q, o, dout) / [N][Hkv_total][d] (k, v)
     const float *lse;
-    void *dq, *dk, *dv;
+    void *dq, *dk, *dv;                 // same row layouts as q / k / v
     int64_t N;
     int Hl, Hkvl, d;
+    int Hq_total, Hkv_total;            // heads per token row (Hl / Hkvl for slice buffers)
+    int q_head0, kv_head0;              // first head of this rank's slice in those rows
     float scale;
     char *ws;
     WsLayout L;

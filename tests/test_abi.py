@@ -91,6 +91,16 @@ def test_attn_argument_errors():
     assert b(*ba(256, 4, 3, 128, FAKE, bws)) == -1
     assert b(*ba(256, 4, 2, 128, FAKE, ws_ok)) == -5              # forward-sized workspace is too small
     assert b(*ba(0, 4, 2, 128, FAKE, bws)) == 0
+    bf = lib.ulysses_attn_bwd_fused
+    bfa = lambda N, P, H, Hkv, rank, wsb: (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, N, P, H, Hkv, 128, rank,
+                                           ctypes.c_float(0.0), FAKE, FAKE, FAKE, FAKE, wsb, None)
+    bws_f = lib.ulysses_attn_workspace_bytes(256, 2, 1, 128, 1)
+    assert bf(*bfa(256, 3, 4, 4, 0, bws_f)) == -1                 # H % P
+    assert bf(*bfa(256, 4, 8, 2, 0, bws_f)) == -1                 # Hkv % P
+    assert bf(*bfa(255, 2, 4, 2, 0, bws_f)) == -1                 # N % P
+    assert bf(*bfa(256, 2, 4, 2, 2, bws_f)) == -1                 # rank
+    assert bf(*bfa(256, 2, 4, 2, 1, bws_f - 1)) == -5             # workspace too small
+    assert bf(*bfa(0, 2, 4, 2, 1, bws_f)) == 0                    # empty
 
 
 def test_python_binding_rejects_cpu_tensors():

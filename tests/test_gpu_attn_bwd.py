@@ -110,3 +110,30 @@ def test_train_workload_documents():
         assert_grad_close(f"dQ doc {t}", bf16_to_f64(dq[sl]), rq)
         assert_grad_close(f"dK doc {t}", bf16_to_f64(dk[sl]), rk)
         assert_grad_close(f"dV doc {t}", bf16_to_f64(dv[sl]), rv)
+
+
+def test_bwd_fused_equals_slice():
+    """The fused backward (reading every rank's head slice straight from the
+    sequence-sharded buffers and writing the gradients back into that layout)
+    gives, bit for bit, the slice backward of each rank: the same kernels on the
+    same values, only the addressing differs."""
+    import long_context_sequence_ulysses_b200 as U
+    lengths = [700, 1, 300, 23]
+    N, P, H, Hkv, d = sum(lengths), 2, 8, 4, 128
+    c = random_case(N, H, Hkv, d, lengths, seed=21, device="cuda", with_grad_out=True)
+    Hl, Hkvl = H // P, Hkv // P
+    dq_f = torch.zeros_like(c["q"]); dk_f = torch.zeros_like(c["k"]); dv_f = torch.zeros_like(c["v"])
+    o_seq = torch.empty_like(c["q"])
+    for r in range(P):
+        qs, ks = slice(r * Hl, (r + 1) * Hl), slice(r * Hkvl, (r + 1) * Hkvl)
+        q, k, v, do = (c["q"][:, qs].contiguous(), c["k"][:, ks].contiguous(), c["v"][:, ks].contiguous(),
+                       c["do"][:, qs].contiguous())
+        o, lse = U.attn_fwd(q, k, v, c["position_ids"])
+        o_seq[:, qs] = o
+        dq, dk, dv = U.attn_bwd(q, k, v, o, do, lse, c["position_ids"])
+        U.attn_bwd_fused(c["q"], c["k"], c["v"], o_seq, c["do"], lse, c["position_ids"], P, r,
+                         dq=dq_f, dk=dk_f, dv=dv_f)
+        torch.cuda.synchronize()
+        assert torch.equal(dq_f[:, qs], dq)
+        assert torch.equal(dk_f[:, ks], dk)
+        assert torch.equal(dv_f[:, ks], dv)
