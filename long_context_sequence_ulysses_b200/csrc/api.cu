@@ -182,7 +182,7 @@ static int attn_fwd_common(const char *name, const void *q, const void *k, const
     if (!aligned4(pos) || !aligned4(lse)) return fail(ULYSSES_ERR_INVALID, "%s: position_ids/lse misaligned", name);
     if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.0f / std::sqrt(static_cast<float>(d));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_docbounds(pos, N, static_cast<char *>(ws), L, false, s);
+    cudaError_t e = launch_docbounds(pos, N, static_cast<char *>(ws), L, false, !fwd_pairs_heads(Hl, Hkvl), s);
     if (e != cudaSuccess) return cuda_fail(e, name);
     FwdLaunch a;
     a.q = q; a.k = k; a.v = v;
@@ -248,7 +248,7 @@ static int attn_bwd_common(const char *name, const void *q, const void *k, const
     if (!aligned4(position_ids) || !aligned4(lse)) return fail(ULYSSES_ERR_INVALID, "%s: position_ids/lse misaligned", name);
     if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.0f / std::sqrt(static_cast<float>(d));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_docbounds(position_ids, N, static_cast<char *>(ws), L, true, s);
+    cudaError_t e = launch_docbounds(position_ids, N, static_cast<char *>(ws), L, true, false, s);
     if (e != cudaSuccess) return cuda_fail(e, name);
     BwdLaunch a;
     a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;

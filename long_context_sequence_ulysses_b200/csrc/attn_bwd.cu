@@ -361,8 +361,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int it = 0; it < n_it; ++it) {
             const int s = it % C::NST, u = it / C::NST;
             const int q0 = (qt0 + it % n_q) * kTileM + part * kPartCols;   // first query of this part
-            if (!mbar_wait(s_full, it & 1, wc)) { ok = false; break; }
-            if (!mbar_wait(&qdo_full[s], u & 1, wc)) { ok = false; break; }
+            // warp-uniform waits: the tcgen05.ld below needs the whole warp converged
+            if (!mbar_wait_warp(s_full, it & 1, wc)) { ok = false; break; }
+            if (!mbar_wait_warp(&qdo_full[s], u & 1, wc)) { ok = false; break; }
             tc_fence_after();
             const float *rl = sRow + (s * 2 + 0) * 128 + part * kPartCols;   // -lse2 of this part's queries
             const float *rd = sRow + (s * 2 + 1) * 128 + part * kPartCols;   // delta of this part's queries
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_before();
             mbar_arrive(p_ready);
             // phase 2: dS^T = P^T (dP^T - D) from the bf16 P^T, bf16 into dP^T's columns
-            if (!mbar_wait(dp_full, it & 1, wc)) { ok = false; break; }
+            if (!mbar_wait_warp(dp_full, it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
                 uint32_t dr[kPartCols];
@@ -424,7 +425,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // ---- epilogue: part p writes d columns [p * E, (p + 1) * E) of dV and dK, E = max(16, D / kParts)
         constexpr int E = (D / kParts) >= 16 ? D / kParts : 16;
-        if (ok && part * E < D && mbar_wait(acc_done, 0, wc)) {
+        if (ok && part * E < D && mbar_wait_warp(acc_done, 0, wc)) {
             tc_fence_after();
             const bool valid = j < p.N;
             const int64_t kv_off = (static_cast<int64_t>(j) * p.Hkv_total + p.kv_head0 + kvh) * D + part * E;
@@ -626,7 +627,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int j = 0; j < n_kv; ++j) {
             const int c0 = (kt0 + j) * kTileN + part * kPartCols;   // first key of this part
             const uint32_t tS = tbase + ((j & 1) ? C::T_S2 : C::T_S) + lane_off + col;
-            if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, wc)) { ok = false; break; }
+            if (!mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
             const bool any_mask = __any_sync(0xffffffffu, (c0 < lo) || (c0 + kPartCols - 1 > i));
             // phase 1 (while dP(j) may still be computing): P = exp2(S * scale*log2(e)
@@ -649,7 +650,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
             // phase 2: dS = P (dP - D) from the bf16 P, bf16 into S's columns
-            if (!mbar_wait(dp_full, j & 1, wc)) { ok = false; break; }
+            if (!mbar_wait_warp(dp_full, j & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
                 uint32_t dr[kPartCols];
@@ -672,7 +673,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // ---- epilogue: part p writes d columns [p * E, (p + 1) * E) of dQ, E = max(16, D / kParts)
         constexpr int E = (D / kParts) >= 16 ? D / kParts : 16;
-        if (ok && part * E < D && mbar_wait(acc_done, 0, wc)) {
+        if (ok && part * E < D && mbar_wait_warp(acc_done, 0, wc)) {
             tc_fence_after();
             __nv_bfloat16 *row = p.dq + (static_cast<int64_t>(i) * p.Hq_total + p.q_head0 + h) * D + part * E;
             const uint32_t tacc = tbase + C::T_ACC0 + lane_off + part * E;

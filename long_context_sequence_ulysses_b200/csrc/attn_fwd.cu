@@ -8,8 +8,13 @@
 // O(n) by tiling with an online softmax (section "超长序列训练的挑战").
 //
 // The kernel is persistent: one CTA per SM takes work items from a global
-// counter, heaviest first. An item is two consecutive 128-row query tiles
-// A = 2u and B = 2u+1 of one head; they share every K/V tile load.
+// counter, heaviest first. An item is two 128-row query tiles A and B that
+// share every K/V tile load. When the query heads of a KV group come in pairs
+// (G = Hl/Hkvl even) they are the same query tile t of heads 2g and 2g+1 of
+// one group: identical key ranges, so both tiles run the same steps.
+// Otherwise (G odd) they are consecutive tiles 2u and 2u+1 of one head; B
+// then has one key tile more than A, and where a document starts inside the
+// pair B's range is much shorter than A's.
 //   warps 0..3   softmax warpgroup of tile A (thread t owns row t = TMEM lane t)
 //   warps 4..7   softmax warpgroup of tile B
 //   warp 8       takes the items and hands them to the other roles through a
@@ -26,8 +31,10 @@
 //     ... PV_A(j-1), S_A(j), PV_B(j-1), S_B(j), PV_A(j), S_A(j+1) ...
 // and runs on into the next item without a break: the K/V rings, the barrier
 // phases and the tensor memory carry over, the next item's Q tiles load as
-// soon as the last S of the current item has read them, and its first S
-// overlaps the current item's epilogue.
+// soon as the last S of the current item has read them, and the step at an
+// item boundary is itself ping-ponged -- PV_A(last), S_A'(0), PV_B(last),
+// S_B'(0) -- so a tile that is done (A has one key tile fewer than B) starts
+// its next item while B finishes, and its first S overlaps its epilogue.
 // S = Q K^T is an SS MMA (both operands K-major in 128B-swizzled shared memory);
 // O += P V is a TS MMA (P from tensor memory, V MN-major from its TMA tile).
 // The softmax reads its S row, masks only diagonal / document-boundary tiles,
@@ -77,15 +84,17 @@ struct FwdParams {
     int N, T, Hl, Hkvl;
     int q_head0, kv_head0;
     float scale_log2;      // softmax scale * log2(e)
-    int items;             // work items: ceil(T / 2) tile pairs x Hl heads
+    int pair_heads;        // 1: items pair heads (T x Hl/2 items); 0: items pair tiles (ceil(T/2) x Hl)
+    int items;
     uint32_t *status;      // [0] status word, [1] work counter (both zeroed before the launch)
     uint64_t wait_limit_ns;
     uint32_t debug_flags;   // bit 0: CTA 0 waits on a barrier nobody arrives on (tests the timeout path)
 };
 
-// One work item: the tile pair q_order[idx / Hl] of head idx % Hl.
+// One work item. Head pairs: tile q_order[idx / (Hl/2)] of heads 2g, 2g+1,
+// g = idx % (Hl/2). Tile pairs: the pair q_order[idx / Hl] of head idx % Hl.
 struct FwdItem {
-    int h, kvh, tA, tB;
+    int hA, hB, kvh, tA, tB;
     bool hasB;
     int j0;        // first key tile of the union of both tiles' ranges
     int nA;        // key tiles of A: union steps [0, nA)
@@ -97,9 +106,22 @@ struct FwdItem {
 __device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
 {
     FwdItem it;
+    if (p.pair_heads) {
+        const int groups2 = p.Hl >> 1;
+        const int t = p.q_order[idx / groups2];
+        it.hA = 2 * (idx % groups2);
+        it.hB = it.hA + 1;
+        it.kvh = it.hA / (p.Hl / p.Hkvl);
+        it.tA = it.tB = t;
+        it.hasB = true;
+        it.j0 = p.tile_lo[t] / kTileN;
+        it.nA = it.nB = it.n_union = t - it.j0 + 1;
+        it.bstart = 0;
+        return it;
+    }
     const int pair = p.q_order[idx / p.Hl];
-    it.h = idx % p.Hl;
-    it.kvh = it.h / (p.Hl / p.Hkvl);
+    it.hA = it.hB = idx % p.Hl;
+    it.kvh = it.hA / (p.Hl / p.Hkvl);
     it.tA = 2 * pair;
     it.tB = 2 * pair + 1;
     it.hasB = it.tB < p.T;
@@ -232,16 +254,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 mbar_arrive(&item_full[slot]);
                 if (idx < 0) break;
                 const FwdItem w = decode_item(p, idx);
-                bool ok = true;
-                for (int x = 0; x < (w.hasB ? 2 : 1); ++x) {
-                    if (qcount[x] > 0 && !mbar_wait(&q_empty[x], (qcount[x] - 1) & 1, wc)) { ok = false; break; }
+                // Q_A, K_0, Q_B, K_1, K_2, ...: the next item's first S (tile A) needs
+                // only Q_A and K_0, and Q_B's buffer is freed last (by B's final S).
+                auto load_q = [&](int x) -> bool {
+                    if (qcount[x] > 0 && !mbar_wait(&q_empty[x], (qcount[x] - 1) & 1, wc)) return false;
                     mbar_arrive_expect_tx(&q_full[x], C::TILE_BYTES);
 #pragma unroll
                     for (int a = 0; a < C::NA; ++a)
                         tma_load_3d(sQ + x * C::TILE_BYTES + a * C::ATOM_BYTES, &tmQ, &q_full[x], a * C::AW,
-                                    p.q_head0 + w.h, (x == 0 ? w.tA : w.tB) * kTileM);
+                                    p.q_head0 + (x == 0 ? w.hA : w.hB), (x == 0 ? w.tA : w.tB) * kTileM);
                     ++qcount[x];
-                }
+                    return true;
+                };
+                bool ok = load_q(0);
                 for (int j = 0; ok && j < w.n_union; ++j, ++kcount) {
                     const int s = kcount % C::KST, u = kcount / C::KST;
                     if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) { ok = false; break; }
@@ -251,6 +276,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmK, &k_full[s], a * C::AW,
                                     p.kv_head0 + w.kvh, (w.j0 + j) * kTileN);
                     last_use[s] = u;
+                    if (j == 0 && w.hasB && !load_q(1)) { ok = false; break; }
                 }
                 if (!ok) break;
             }
@@ -317,63 +343,121 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 umma_ts_elect_off(tbase + C::to_col(x), tbase + C::ts_col(x) + kk * 8, bd, (kk * 16 * C::SW) >> 4,
                                   C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
         };
-        int kbase = 0, vbase = 0;            // K / V tiles consumed by earlier items
+        int kbase = 0, vbase = 0;            // K / V ring positions of the current item's first tile
         int pbase[2] = {0, 0};               // P tiles of each tile slot consumed by earlier items
         int qcount[2] = {0, 0};
         bool ok = true;
+        FwdItem cur{};
+        bool have_cur = false;
         for (int n = 0; ok; ++n) {
+            // ---- boundary step: the last PVs of the current item, interleaved per
+            // tile with the first S of item n, so that a tile that has finished
+            // starts its next item without waiting for the other tile's last step:
+            //     PV_A(cur, last), S_A(next, 0), PV_B(cur, last), S_B(next, 0)
             const int idx = take_item(n, true);
             if (lane == 0) mbar_arrive(&item_empty[n & 1]);
             __syncwarp();
-            if (idx < 0) break;
-            const FwdItem w = decode_item(p, idx);
-            ok = mbar_wait_warp(&q_full[0], qcount[0] & 1, wc);
-            if (ok && w.hasB) ok = mbar_wait_warp(&q_full[1], qcount[1] & 1, wc);
-            for (int j = 0; ok && j <= w.n_union; ++j) {
-                const int gk = kbase + j, gv = vbase + j - 1;   // ring positions of K_j and V_(j-1)
-                const int s = gk % C::KST, u = gk / C::KST;
-                const int sp = (gv + C::VST) % C::VST, up = gv / C::VST;
-                const bool have_j = j < w.n_union;
-                const bool pvA = (j - 1 >= 0) && (j - 1 < w.nA);
-                const bool sA = have_j && j < w.nA;
-                const int jb = j - w.bstart;
-                const bool pvB = w.hasB && (jb - 1 >= 0) && (jb - 1 < w.nB);
-                const bool sB = w.hasB && have_j && jb >= 0 && jb < w.nB;
-                if ((pvA || pvB) && !mbar_wait_warp(&v_full[sp], up & 1, wc)) { ok = false; break; }
-                if ((sA || sB) && !mbar_wait_warp(&k_full[s], u & 1, wc)) { ok = false; break; }
-                // tile A
-                if (pvA) {
-                    if (!mbar_wait_warp(&p_full[0], (pbase[0] + j - 1) & 1, wc)) { ok = false; break; }
+            const bool have_nxt = idx >= 0;
+            FwdItem nxt{};
+            if (have_nxt) nxt = decode_item(p, idx);
+            const int nu = have_cur ? cur.n_union : 0;
+            const int gv = vbase + nu - 1;                     // V position of the current item's last PV
+            const int sp = (gv + C::VST) % C::VST, up = gv / C::VST;
+            const int gk = kbase + nu;                         // K position of the next item's first S
+            const int s = gk % C::KST, u = gk / C::KST;
+            // A tile's last PV falls on the boundary when its key range ends the
+            // union; B's always does (its range ends at its own diagonal tile).
+            const bool pvA = have_cur && cur.nA == nu;
+            const bool pvB = have_cur && cur.hasB;
+            const bool sA = have_nxt;
+            const bool sB = have_nxt && nxt.hasB && nxt.bstart == 0;
+            if (pvA || pvB) ok = mbar_wait_warp(&v_full[sp], up & 1, wc);
+            if (ok && sA) ok = mbar_wait_warp(&k_full[s], u & 1, wc);
+            if (ok && pvA) {
+                ok = mbar_wait_warp(&p_full[0], (pbase[0] + cur.nA - 1) & 1, wc);
+                if (ok) {
                     tc_fence_after();
-                    issue_pv(0, sp, j - 1 == 0);
-                    if (j - 1 == w.nA - 1) umma_commit_elect(&o_done[0]);
+                    issue_pv(0, sp, cur.nA == 1);
+                    umma_commit_elect(&o_done[0]);
                 }
-                if (sA) {
+            }
+            if (ok && sA) {
+                ok = mbar_wait_warp(&q_full[0], qcount[0] & 1, wc);
+                ++qcount[0];
+                if (ok) {
                     tc_fence_after();
                     issue_s(0, s);
-                    if (j == w.nA - 1) umma_commit_elect(&q_empty[0]);
+                    if (nxt.nA == 1) umma_commit_elect(&q_empty[0]);
+                }
+            }
+            if (ok && pvB) {
+                ok = mbar_wait_warp(&p_full[1], (pbase[1] + cur.nB - 1) & 1, wc);
+                if (ok) {
+                    tc_fence_after();
+                    issue_pv(1, sp, cur.nB == 1);
+                    umma_commit_elect(&o_done[1]);
+                }
+            }
+            if (ok && have_nxt && nxt.hasB) {
+                ok = mbar_wait_warp(&q_full[1], qcount[1] & 1, wc);
+                ++qcount[1];
+            }
+            if (ok && sB) {
+                tc_fence_after();
+                issue_s(1, s);
+                if (nxt.nB == 1) umma_commit_elect(&q_empty[1]);
+            }
+            if (!ok) break;
+            if (sA) umma_commit_elect(&k_empty[s]);
+            if (pvA || pvB) umma_commit_elect(&v_empty[sp]);
+            if (have_cur) {
+                kbase += cur.n_union;
+                vbase += cur.n_union;
+                pbase[0] += cur.nA;
+                pbase[1] += cur.nB;
+            }
+            if (!have_nxt) break;
+            cur = nxt;
+            have_cur = true;
+            // ---- steps 1 .. n_union-1 of the item: PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)
+            for (int j = 1; ok && j < cur.n_union; ++j) {
+                const int gkj = kbase + j, gvj = vbase + j - 1;   // ring positions of K_j and V_(j-1)
+                const int sj = gkj % C::KST, uj = gkj / C::KST;
+                const int spj = gvj % C::VST, upj = gvj / C::VST;
+                const bool pvAj = j - 1 < cur.nA;
+                const bool sAj = j < cur.nA;
+                const int jb = j - cur.bstart;
+                const bool pvBj = cur.hasB && jb - 1 >= 0 && jb - 1 < cur.nB;
+                const bool sBj = cur.hasB && jb >= 0 && jb < cur.nB;
+                if ((pvAj || pvBj) && !mbar_wait_warp(&v_full[spj], upj & 1, wc)) { ok = false; break; }
+                if ((sAj || sBj) && !mbar_wait_warp(&k_full[sj], uj & 1, wc)) { ok = false; break; }
+                // tile A
+                if (pvAj) {
+                    if (!mbar_wait_warp(&p_full[0], (pbase[0] + j - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(0, spj, j - 1 == 0);
+                    if (j - 1 == cur.nA - 1) umma_commit_elect(&o_done[0]);
+                }
+                if (sAj) {
+                    tc_fence_after();
+                    issue_s(0, sj);
+                    if (j == cur.nA - 1) umma_commit_elect(&q_empty[0]);
                 }
                 // tile B
-                if (pvB) {
+                if (pvBj) {
                     if (!mbar_wait_warp(&p_full[1], (pbase[1] + jb - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(1, sp, jb - 1 == 0);
-                    if (jb - 1 == w.nB - 1) umma_commit_elect(&o_done[1]);
+                    issue_pv(1, spj, jb - 1 == 0);
+                    if (jb - 1 == cur.nB - 1) umma_commit_elect(&o_done[1]);
                 }
-                if (sB) {
+                if (sBj) {
                     tc_fence_after();
-                    issue_s(1, s);
-                    if (jb == w.nB - 1) umma_commit_elect(&q_empty[1]);
+                    issue_s(1, sj);
+                    if (jb == cur.nB - 1) umma_commit_elect(&q_empty[1]);
                 }
-                if (sA || sB) umma_commit_elect(&k_empty[s]);
-                if (pvA || pvB) umma_commit_elect(&v_empty[sp]);
+                if (sAj || sBj) umma_commit_elect(&k_empty[sj]);
+                if (pvAj || pvBj) umma_commit_elect(&v_empty[spj]);
             }
-            kbase += w.n_union;
-            vbase += w.n_union;
-            pbase[0] += w.nA;
-            pbase[1] += w.nB;
-            ++qcount[0];
-            if (w.hasB) ++qcount[1];
         }
         umma_commit_elect(mma_done);
         WaitCtx drain{p.wait_limit_ns, p.status, false};
@@ -391,7 +475,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         int sbase = 0;      // S tiles of this slot consumed by earlier items
         int ocount = 0;     // items finished by this slot
         bool ok = true;
-        if ((p.debug_flags & 1u) && blockIdx.x == 0 && x == 0) ok = mbar_wait(never, 0, wc);   // runs out
+        if ((p.debug_flags & 1u) && blockIdx.x == 0 && x == 0) ok = mbar_wait_warp(never, 0, wc);   // runs out
         for (int n = 0; ok; ++n) {
             const int idx = take_item(n, false);
             mbar_arrive(&item_empty[n & 1]);
@@ -400,6 +484,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int n_it = x == 0 ? w.nA : w.nB;
             if (n_it == 0) continue;
             const int first_union = x == 0 ? 0 : w.bstart;
+            const int hx = x == 0 ? w.hA : w.hB;
             const int i = (x == 0 ? w.tA : w.tB) * kTileM + r;
             const bool valid = i < p.N;
             const int lo = valid ? p.doc_start[i] : i;
@@ -407,7 +492,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             float ms = -CUDART_INF_F;   // exponent offset in use (scaled log2 units)
             float l = 0.f;
             for (int it = 0; it < n_it; ++it) {
-                if (!mbar_wait(&s_full[x], (sbase + it) & 1, wc)) { ok = false; break; }
+                // warp-uniform wait: the tcgen05.ld below needs the whole warp converged
+                if (!mbar_wait_warp(&s_full[x], (sbase + it) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 float s[kTileN];
                 {
@@ -442,10 +528,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         }
                     }
                 }
-                // row max: 4 independent chains of 3-input max
-                float mx[4] = {s[0], s[1], s[2], s[3]};
+                // row max: 4 independent chains of 3-input max, column groups of 8
+                static_assert(kTileN % 8 == 0, "row max works on groups of 8 columns");
+                float mx[4];
 #pragma unroll
-                for (int c = 4; c < kTileN; c += 8)
+                for (int e = 0; e < 4; ++e) mx[e] = fmaxf(s[e], s[4 + e]);
+#pragma unroll
+                for (int c = 8; c < kTileN; c += 8)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) mx[e] = max3f(mx[e], s[c + e], s[c + 4 + e]);
                 const float mt = row_out ? -CUDART_INF_F : max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
@@ -501,12 +590,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             sbase += n_it;
             // ---- epilogue: O / l -> bf16, LSE. The next item's first PV into O_x
             // waits for this slot's next P, which comes after these reads.
-            if (!ok || !mbar_wait(&o_done[x], ocount & 1, wc)) { ok = false; break; }
+            if (!ok || !mbar_wait_warp(&o_done[x], ocount & 1, wc)) { ok = false; break; }
             ++ocount;
             tc_fence_after();
             const float inv_l = 1.f / l;
             __nv_bfloat16 *orow = p.o + static_cast<int64_t>(i) * p.o_row_elems +
-                                  static_cast<int64_t>(p.o_head0 + w.h) * D;
+                                  static_cast<int64_t>(p.o_head0 + hx) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t raw[32];
@@ -523,7 +612,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
                 }
             }
-            if (valid) p.lse[static_cast<int64_t>(w.h) * p.N + i] = (ms + __log2f(l)) * 0.69314718055994530942f;
+            if (valid) p.lse[static_cast<int64_t>(hx) * p.N + i] = (ms + __log2f(l)) * 0.69314718055994530942f;
             tc_fence_before();
         }
     }
@@ -564,7 +653,8 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.kv_head0 = a.kv_head0;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.status = reinterpret_cast<uint32_t *>(const_cast<char *>(a.ws) + a.L.status);
-    p.items = static_cast<int>(ceil_div(p.T, 2) * a.Hl);
+    p.pair_heads = fwd_pairs_heads(a.Hl, a.Hkvl) ? 1 : 0;
+    p.items = p.pair_heads ? static_cast<int>(p.T * (a.Hl / 2)) : static_cast<int>(ceil_div(p.T, 2) * a.Hl);
     p.wait_limit_ns = a.wait_limit_ns;
     p.debug_flags = a.debug_flags;
     static bool attr_set[64] = {};

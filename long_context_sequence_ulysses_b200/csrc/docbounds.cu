@@ -13,8 +13,10 @@
 // Kernels: a block-local scan, a fix-up with the carry of earlier blocks
 // (which also writes each query tile's first key), for the backward the last
 // query row of each key tile (a binary search over doc_start), and a counting
-// sort of the scheduling units (pairs of query tiles for the forward, key
-// tiles for the backward) by work, heaviest first.
+// sort of the scheduling units by work, heaviest first: query tiles (the
+// backward, and a forward whose items pair two heads of one KV group), pairs
+// of consecutive query tiles (a forward with an odd group size), and key
+// tiles (the backward).
 #include "ulysses_internal.cuh"
 
 namespace uly {
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(1024) unit_order_kernel(int units, int T, int 
 }  // namespace
 
 cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
-                             cudaStream_t stream)
+                             bool fwd_tile_pairs, cudaStream_t stream)
 {
     const int64_t T = ceil_div(N, kTileM);
     const int nb = static_cast<int>(ceil_div(N, kScanBlock));
@@ -181,7 +183,7 @@ cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLa
     doc_scan_kernel<<<nb, kScanBlock, 0, stream>>>(pos, N, doc_start, block_agg,
                                                    reinterpret_cast<uint32_t *>(ws + L.status));
     doc_fixup_kernel<<<nb, kScanBlock, 0, stream>>>(N, doc_start, block_agg, tile_lo);
-    if (!backward) {
+    if (!backward && fwd_tile_pairs) {
         const int pairs = static_cast<int>(ceil_div(T, 2));
         unit_order_kernel<Unit::kQueryPairs><<<1, 1024, 0, stream>>>(pairs, static_cast<int>(T),
                                                                      static_cast<int>(2 * T), tile_lo, scratch,
@@ -190,6 +192,8 @@ cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLa
         unit_order_kernel<Unit::kQueryTiles><<<1, 1024, 0, stream>>>(static_cast<int>(T), static_cast<int>(T),
                                                                      static_cast<int>(T), tile_lo, scratch,
                                                                      reinterpret_cast<int32_t *>(ws + L.q_order));
+    }
+    if (backward) {
         int32_t *kv_qend = reinterpret_cast<int32_t *>(ws + L.kv_qend);
         kv_qend_kernel<<<static_cast<int>(ceil_div(T, 256)), 256, 0, stream>>>(N, static_cast<int>(T), doc_start,
                                                                                kv_qend);

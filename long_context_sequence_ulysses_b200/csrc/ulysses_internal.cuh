@@ -21,8 +21,9 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 //                                 [1] work counter of the persistent forward kernel
 //   doc_start  int32  [N]         first token of the row's document
 //   tile_lo    int32  [T]         doc_start of the first row of each 128-row tile
-//   q_order    int32  [T]         forward: pairs of query tiles (2u, 2u+1), heaviest
-//                                 first; backward: single query tiles, heaviest first
+//   q_order    int32  [T]         query tiles heaviest first (backward, and the
+//                                 forward when its items pair heads); forward with
+//                                 tile-pair items: pairs (2u, 2u+1), heaviest first
 //   block_agg  int32  [ceil(N/1024)]  per-block maxima of the doc-start scan
 //   scratch    int32  [2T + 2]    histogram for the tile sort
 // backward only (Npad = T * 128):
@@ -64,10 +65,15 @@ inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
 cudaError_t launch_relayout(bool to_head, const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
                             cudaStream_t stream, int num_sms);
 
-// docbounds.cu: doc_start, tile_lo and the query order (pairs of tiles for the
-// forward; single tiles, kv_qend and the key-tile order for the backward).
+// The forward pairs two query heads of one KV group in a work item when the
+// group size Hl/Hkvl is even, else two consecutive query tiles of one head.
+inline bool fwd_pairs_heads(int Hl, int Hkvl) { return Hkvl > 0 && (Hl / Hkvl) % 2 == 0; }
+
+// docbounds.cu: doc_start, tile_lo and the query order (single tiles, or
+// pairs of tiles for a forward with tile-pair items; for the backward also
+// kv_qend and the key-tile order).
 cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
-                             cudaStream_t stream);   // also clears the status word
+                             bool fwd_tile_pairs, cudaStream_t stream);   // also clears the status word
 
 // Forward attention launch description.
 struct FwdLaunch {

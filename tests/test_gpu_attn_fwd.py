@@ -37,6 +37,8 @@ CASES = [
     ([513, 511], 4, 4, 32),
     ([2048], 1, 1, 64),
     ([3000, 1500, 2], 2, 1, 128),
+    ([600, 700, 29], 6, 2, 64),       # odd group size: items pair consecutive tiles
+    ([1100, 3], 3, 1, 128),
 ]
 
 
