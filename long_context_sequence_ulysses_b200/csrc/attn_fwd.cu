@@ -91,11 +91,14 @@ struct FwdParams {
     uint32_t debug_flags;   // bit 0: CTA 0 waits on a barrier nobody arrives on (tests the timeout path)
 };
 
+constexpr int kItemInts = 12;   // ints of one FwdItem
+
 // One work item. Head pairs: tile q_order[idx / (Hl/2)] of heads 2g, 2g+1,
 // g = idx % (Hl/2). Tile pairs: the pair q_order[idx / Hl] of head idx % Hl.
 struct FwdItem {
+    int idx;       // work item index, -1: no more work
     int hA, hB, kvh, tA, tB;
-    bool hasB;
+    int hasB;
     int j0;        // first key tile of the union of both tiles' ranges
     int nA;        // key tiles of A: union steps [0, nA)
     int bstart;    // key tiles of B: union steps [bstart, n_union)
@@ -106,6 +109,7 @@ struct FwdItem {
 __device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
 {
     FwdItem it;
+    it.idx = idx;
     if (p.pair_heads) {
         const int groups2 = p.Hl >> 1;
         const int t = p.q_order[idx / groups2];
@@ -113,7 +117,7 @@ __device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
         it.hB = it.hA + 1;
         it.kvh = it.hA / (p.Hl / p.Hkvl);
         it.tA = it.tB = t;
-        it.hasB = true;
+        it.hasB = 1;
         it.j0 = p.tile_lo[t] / kTileN;
         it.nA = it.nB = it.n_union = t - it.j0 + 1;
         it.bstart = 0;
@@ -124,7 +128,7 @@ __device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
     it.kvh = it.hA / (p.Hl / p.Hkvl);
     it.tA = 2 * pair;
     it.tB = 2 * pair + 1;
-    it.hasB = it.tB < p.T;
+    it.hasB = it.tB < p.T ? 1 : 0;
     it.j0 = p.tile_lo[it.tA] / kTileN;
     it.nA = it.tA - it.j0 + 1;
     const int loB = it.hasB ? p.tile_lo[it.tB] / kTileN : 0;
@@ -149,7 +153,7 @@ struct FwdCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     static constexpr int NBAR = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 2 + 2 + 1 + 1;
-    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 16 + 1024;   // + item ring, alignment slack
+    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 2 * kItemInts * 4 + 1024;   // + item ring, alignment slack
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kTileM, kTileN, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kTileM, D, false, true);
     // tensor-memory columns: S / P of tile x at ts_col(x), O of tile x at to_col(x)
@@ -183,7 +187,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t *mma_done = item_empty + 2;
     uint64_t *never = mma_done + 1;          // never arrived on (timeout test only)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(never + 1);
-    volatile int *item_ring = reinterpret_cast<volatile int *>(tmem_holder + 4);   // [2]
+    // two decoded FwdItems, written by the producer, read by every other role
+    volatile int *item_ring = reinterpret_cast<volatile int *>(tmem_holder + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -224,13 +229,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // A CTA that starts after another one has timed out skips its work.
     WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
 
-    // Consumer side of the item ring: the n-th item of this CTA (-1: no more work).
-    auto take_item = [&](int n, bool warp_wide) -> int {
+    // Consumer side of the item ring: the n-th item of this CTA, decoded by the
+    // producer (idx -1: no more work).
+    auto take_item = [&](int n, bool warp_wide) -> FwdItem {
         const int slot = n & 1;
         const bool ok = warp_wide ? mbar_wait_warp(&item_full[slot], (n >> 1) & 1, wc)
                                   : mbar_wait(&item_full[slot], (n >> 1) & 1, wc);
-        if (!ok) return -1;
-        return item_ring[slot];
+        FwdItem w;
+        int *wi = reinterpret_cast<int *>(&w);
+#pragma unroll
+        for (int f = 0; f < kItemInts; ++f) wi[f] = item_ring[slot * kItemInts + f];
+        if (!ok) w.idx = -1;
+        return w;
     };
 
     if (warp >= 8) {
@@ -248,12 +258,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int n = 0;; ++n) {
                 const int slot = n & 1;
                 if (n >= 2 && !mbar_wait(&item_empty[slot], ((n >> 1) - 1) & 1, wc)) break;
-                int idx = static_cast<int>(atomicAdd(p.status + 1, 1u));
-                if (idx >= p.items) idx = -1;
-                item_ring[slot] = idx;
-                mbar_arrive(&item_full[slot]);
-                if (idx < 0) break;
-                const FwdItem w = decode_item(p, idx);
+                const int idx = static_cast<int>(atomicAdd(p.status + 1, 1u));
+                FwdItem w{};
+                w.idx = -1;
+                if (idx < p.items) w = decode_item(p, idx);
+                const int *wi = reinterpret_cast<const int *>(&w);
+#pragma unroll
+                for (int f = 0; f < kItemInts; ++f) item_ring[slot * kItemInts + f] = wi[f];
+                mbar_arrive(&item_full[slot]);   // release: the fields are visible to every waiter
+                if (w.idx < 0) break;
                 // Q_A, K_0, Q_B, K_1, K_2, ...: the next item's first S (tile A) needs
                 // only Q_A and K_0, and Q_B's buffer is freed last (by B's final S).
                 auto load_q = [&](int x) -> bool {
@@ -296,10 +309,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int s = 0; s < C::VST; ++s) last_use[s] = -1;
             for (int n = 0;; ++n) {
-                const int idx = take_item(n, false);
+                const FwdItem w = take_item(n, false);
                 mbar_arrive(&item_empty[n & 1]);
-                if (idx < 0) break;
-                const FwdItem w = decode_item(p, idx);
+                if (w.idx < 0) break;
                 bool ok = true;
                 for (int j = 0; j < w.n_union; ++j, ++vcount) {
                     const int s = vcount % C::VST, u = vcount / C::VST;
@@ -354,12 +366,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // tile with the first S of item n, so that a tile that has finished
             // starts its next item without waiting for the other tile's last step:
             //     PV_A(cur, last), S_A(next, 0), PV_B(cur, last), S_B(next, 0)
-            const int idx = take_item(n, true);
+            const FwdItem nxt = take_item(n, true);
             if (lane == 0) mbar_arrive(&item_empty[n & 1]);
             __syncwarp();
-            const bool have_nxt = idx >= 0;
-            FwdItem nxt{};
-            if (have_nxt) nxt = decode_item(p, idx);
+            const bool have_nxt = nxt.idx >= 0;
             const int nu = have_cur ? cur.n_union : 0;
             const int gv = vbase + nu - 1;                     // V position of the current item's last PV
             const int sp = (gv + C::VST) % C::VST, up = gv / C::VST;
@@ -477,10 +487,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bool ok = true;
         if ((p.debug_flags & 1u) && blockIdx.x == 0 && x == 0) ok = mbar_wait_warp(never, 0, wc);   // runs out
         for (int n = 0; ok; ++n) {
-            const int idx = take_item(n, false);
+            const FwdItem w = take_item(n, false);
             mbar_arrive(&item_empty[n & 1]);
-            if (idx < 0) break;
-            const FwdItem w = decode_item(p, idx);
+            if (w.idx < 0) break;
             const int n_it = x == 0 ? w.nA : w.nB;
             if (n_it == 0) continue;
             const int first_union = x == 0 ? 0 : w.bstart;
@@ -596,15 +605,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const float inv_l = 1.f / l;
             __nv_bfloat16 *orow = p.o + static_cast<int64_t>(i) * p.o_row_elems +
                                   static_cast<int64_t>(p.o_head0 + hx) * D;
+            // the whole O row in one round trip (up to two x64 loads, one wait)
+            uint32_t orw[D];
+            if constexpr (D >= 64) {
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+                    tmem_ld64(tO + c * 64, *reinterpret_cast<uint32_t(*)[64]>(orw + c * 64));
+            } else {
+                tmem_ld32(tO, *reinterpret_cast<uint32_t(*)[32]>(orw));
+            }
+            tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t raw[32];
-                tmem_ld32(tO + c * 32, raw);
-                tmem_ld_wait();
                 uint32_t wv[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    wv[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l, __uint_as_float(raw[2 * e + 1]) * inv_l);
+                    wv[e] = pack_bf16x2(__uint_as_float(orw[c * 32 + 2 * e]) * inv_l,
+                                        __uint_as_float(orw[c * 32 + 2 * e + 1]) * inv_l);
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
