@@ -122,14 +122,50 @@ __device__ __forceinline__ int unit_work(int t, int T, const int32_t *__restrict
     return w;
 }
 
+// Exclusive prefix sum over the 1024 threads of a block (warp shuffles, then
+// the 32 warp totals in warp 0). warp_tot: 32 ints of shared memory.
+__device__ __forceinline__ int block_excl_sum_1024(int v, int *warp_tot)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += u;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += u;
+        }
+        warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int r = (warp > 0 ? warp_tot[warp - 1] : 0) + x - v;
+    __syncthreads();   // warp_tot may be reused after this
+    return r;
+}
+
+// Largest work value whose histogram is kept in shared memory.
+constexpr int kOrderSmemWork = 11999;   // 48 KB of static shared memory with warp_tot
+
 // Counting sort of `units` scheduling units by work (in [0, max_work]),
-// heaviest first. One CTA; hist lives in global scratch [max_work + 1].
+// heaviest first. One CTA of 1024 threads; the histogram lives in shared
+// memory up to kOrderSmemWork, else in global scratch [max_work + 1]. Units
+// of equal work are placed in arrival order of the atomics (any order is a
+// valid schedule).
 template <Unit kUnit>
 __global__ void __launch_bounds__(1024) unit_order_kernel(int units, int T, int max_work,
                                                          const int32_t *__restrict__ src,
-                                                         int32_t *__restrict__ hist, int32_t *__restrict__ order)
+                                                         int32_t *__restrict__ ghist, int32_t *__restrict__ order)
 {
-    __shared__ int part[1024];
+    __shared__ int shist[kOrderSmemWork + 1];
+    __shared__ int warp_tot[32];
+    int *hist = max_work <= kOrderSmemWork ? shist : ghist;
     const int tid = threadIdx.x;
     for (int w = tid; w <= max_work; w += 1024) hist[w] = 0;
     __syncthreads();
@@ -145,15 +181,7 @@ __global__ void __launch_bounds__(1024) unit_order_kernel(int units, int T, int 
         const int w = hi - k;
         if (w >= 0) sum += hist[w];
     }
-    part[tid] = sum;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        const int add = tid >= o ? part[tid - o] : 0;
-        __syncthreads();
-        part[tid] += add;
-        __syncthreads();
-    }
-    int run = part[tid] - sum;   // units with work above this segment
+    int run = block_excl_sum_1024(sum, warp_tot);   // units with work above this segment
     for (int k = 0; k < per; ++k) {
         const int w = hi - k;
         if (w >= 0) {
