@@ -39,6 +39,8 @@ CASES = [
     ([3000, 1500, 2], 2, 1, 128),
     ([600, 700, 29], 6, 2, 64),       # odd group size: items pair consecutive tiles
     ([1100, 3], 3, 1, 128),
+    ([900, 100, 44], 8, 1, 64),       # group of 8: four head pairs share each K/V tile
+    ([600, 33], 2, 1, 32),            # head pairs with the smallest head dimension
 ]
 
 
