@@ -17,9 +17,9 @@
 // pair B's range is much shorter than A's.
 //   warps 0..3   softmax warpgroup of tile A (thread t owns row t = TMEM lane t)
 //   warps 4..7   softmax warpgroup of tile B
-//   warp 8       takes the items and hands them to the other roles through a
-//                two-slot ring in shared memory; TMA producer of Q_A, Q_B and
-//                of the K tiles (KST-stage ring)
+//   warp 8       takes the items, decodes them and hands them to the other
+//                roles through a two-slot ring in shared memory; TMA producer
+//                of Q_A, K_0, Q_B, K_1, ... (K in a KST-stage ring)
 //   warp 9       allocates tensor memory; issues every tcgen05.mma (one elected lane)
 //   warp 10      TMA producer of the V tiles (VST-stage ring; a V tile is held one
 //                step longer than its K tile, so it gets the extra stage)
@@ -33,8 +33,9 @@
 // phases and the tensor memory carry over, the next item's Q tiles load as
 // soon as the last S of the current item has read them, and the step at an
 // item boundary is itself ping-ponged -- PV_A(last), S_A'(0), PV_B(last),
-// S_B'(0) -- so a tile that is done (A has one key tile fewer than B) starts
-// its next item while B finishes, and its first S overlaps its epilogue.
+// S_B'(0) -- so a tile that is done starts its next item without waiting for
+// the other tile's last step, and its first S overlaps its epilogue.
+// Waits before a .sync.aligned tensor-memory load are warp-uniform.
 // S = Q K^T is an SS MMA (both operands K-major in 128B-swizzled shared memory);
 // O += P V is a TS MMA (P from tensor memory, V MN-major from its TMA tile).
 // The softmax reads its S row, masks only diagonal / document-boundary tiles,
@@ -67,8 +68,8 @@ constexpr uint32_t kTmemCols = 512;
 // (2 of 8 measured fastest: 2% over 3 of 8, 6% over 4 of 8).
 constexpr int kEmuPairs = 2;
 // Register split: launched at 168 per thread (384 x 168 = 64512); the two
-// softmax warpgroups take 224, the producer / MMA warpgroup keeps 56:
-// 256 x 224 + 128 x 56 = 64512.
+// softmax warpgroups take 216, the producer / MMA warpgroup keeps 72:
+// 256 x 216 + 128 x 72 = 64512.
 constexpr uint32_t kLaunchRegs = 168;
 constexpr uint32_t kSoftmaxRegs = 216;
 constexpr uint32_t kControlRegs = 72;
@@ -106,6 +107,7 @@ struct FwdItem {
     int nB;
     int n_union;
 };
+static_assert(sizeof(FwdItem) == kItemInts * sizeof(int), "the item ring copies a FwdItem as kItemInts ints");
 
 __device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
 {
