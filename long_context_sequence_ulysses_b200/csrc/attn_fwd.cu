@@ -674,7 +674,9 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.status = reinterpret_cast<uint32_t *>(const_cast<char *>(a.ws) + a.L.status);
     p.pair_heads = fwd_pairs_heads(a.Hl, a.Hkvl) ? 1 : 0;
-    p.items = p.pair_heads ? static_cast<int>(p.T * (a.Hl / 2)) : static_cast<int>(ceil_div(p.T, 2) * a.Hl);
+    const int64_t items = p.pair_heads ? int64_t(p.T) * (a.Hl / 2) : ceil_div(p.T, 2) * a.Hl;
+    if (items > INT32_MAX) return cudaErrorInvalidValue;   // the work counter and item indices are 32-bit
+    p.items = static_cast<int>(items);
     p.wait_limit_ns = a.wait_limit_ns;
     p.debug_flags = a.debug_flags;
     static bool attr_set[64] = {};
