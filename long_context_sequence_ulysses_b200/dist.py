@@ -103,3 +103,61 @@ def attention_forward(q_local: torch.Tensor, k_local: torch.Tensor, v_local: tor
         attn = U.attn_fwd
     o, lse = attn(q, k, v, pos, scale=scale)
     return head_to_seq(o, group, unpack), lse, pos
+
+
+def attention_forward_chunked(q_local: torch.Tensor, k_local: torch.Tensor, v_local: torch.Tensor,
+                              pos_local: torch.Tensor, chunks: int, group=None, scale: Optional[float] = None,
+                              attn: Optional[Callable] = None, pack=None, unpack=None):
+    """The Ulysses attention step of one rank with the heads taken in
+    ``chunks`` groups, the head-chunked variant the pages list as UPipe (page
+    "Ulysses 序列並行：百萬 Token 上下文訓練", section "競品分析"): chunk c's Q/K/V
+    cross the first all-to-all while chunk c-1 is being computed, and only
+    one chunk's head slices are resident at a time, so the activation memory
+    of the exchange and of the attention inputs shrinks by ``chunks``.
+
+    Chunk c holds query heads [c*H/chunks, (c+1)*H/chunks) and KV heads
+    [c*Hkv/chunks, (c+1)*Hkv/chunks); each rank gets 1/G of both, which keeps
+    every query head with its KV head as long as Hkv is divisible by
+    chunks*G. Returns (o_local [N/G][H][d], lse [chunks][H/(chunks*G)][N],
+    position ids of the whole sequence, heads) where heads[c][j] is the
+    global query head of lse[c][j]."""
+    G, rank = _world(group)
+    n_loc, H, d = q_local.shape
+    Hkv = k_local.shape[1]
+    if chunks < 1 or H % (chunks * G) or Hkv % (chunks * G):
+        raise ValueError(f"H={H} and Hkv={Hkv} must be divisible by chunks*G={chunks * G}")
+    if n_loc % G:
+        raise ValueError(f"local tokens ({n_loc}) must be divisible by the group size {G}")
+    Hc, Hkvc = H // chunks, Hkv // chunks
+    if attn is None:
+        import long_context_sequence_ulysses_b200 as U
+        attn = U.attn_fwd
+    pos = gather_position_ids(pos_local, group)
+
+    def start(c: int):
+        """Pack chunk c's Q, K, V and start their all-to-alls (asynchronous)."""
+        inflight = []
+        for x, h in ((q_local, Hc), (k_local, Hkvc), (v_local, Hkvc)):
+            xc = x[:, c * h:(c + 1) * h].contiguous()
+            send = _cuda_pack(xc, G) if pack is None else pack(xc, G)   # [G][N/G][h/G][d]
+            send = send.contiguous()
+            recv = torch.empty_like(send)
+            work = dist.all_to_all_single(recv.view(torch.uint8), send.view(torch.uint8), group=group,
+                                          async_op=True)
+            inflight.append((work, recv, send))
+        return inflight
+
+    o_local = torch.empty_like(q_local)
+    lses, heads = [], []
+    pending = start(0)
+    for c in range(chunks):
+        current = pending
+        pending = start(c + 1) if c + 1 < chunks else None
+        for work, _, _ in current:
+            work.wait()
+        q, k, v = (recv.view(G * n_loc, recv.shape[2], d) for _, recv, _ in current)
+        o, lse = attn(q, k, v, pos, scale=scale)
+        o_local[:, c * Hc:(c + 1) * Hc] = head_to_seq(o, group, unpack)
+        lses.append(lse)
+        heads.append([c * Hc + rank * (Hc // G) + j for j in range(Hc // G)])
+    return o_local, torch.stack(lses), pos, heads

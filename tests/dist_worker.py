@@ -23,7 +23,7 @@ def worker(rank: int, world: int, port: int, case: dict, out_q):
     try:
         _run(rank, world, case, out_q)
     except Exception as e:  # report instead of leaving the parent waiting
-        out_q.put((rank, "error", repr(e), None))
+        out_q.put((rank, "error", repr(e), None, None))
         raise
     finally:
         dist.destroy_process_group()
@@ -52,8 +52,15 @@ def _run(rank, world, case, out_q):
             o, lse = oracle.attn_fwd(q, k, v, pos, scale=scale)
             return torch.from_numpy(o).to(torch.bfloat16), torch.from_numpy(lse)
 
-        o_loc, lse, pos = udist.attention_forward(c["q"][sl].contiguous(), c["k"][sl].contiguous(),
-                                                  c["v"][sl].contiguous(), c["position_ids"][sl].contiguous(),
-                                                  attn=attn, pack=pack, unpack=unpack)
-        out_q.put((rank, o_loc.view(torch.int16).numpy().copy(), lse.numpy().copy(), pos.numpy().copy()))
+        args = (c["q"][sl].contiguous(), c["k"][sl].contiguous(), c["v"][sl].contiguous(),
+                c["position_ids"][sl].contiguous())
+        if case.get("chunks"):
+            o_loc, lse, pos, heads = udist.attention_forward_chunked(*args, case["chunks"], attn=attn, pack=pack,
+                                                                     unpack=unpack)
+            lse = lse.reshape(-1, N)
+            heads = np.array([h for hc in heads for h in hc])
+        else:
+            o_loc, lse, pos = udist.attention_forward(*args, attn=attn, pack=pack, unpack=unpack)
+            heads = np.arange(rank * (case["H"] // world), (rank + 1) * (case["H"] // world))
+        out_q.put((rank, o_loc.view(torch.int16).numpy().copy(), lse.numpy().copy(), pos.numpy().copy(), heads))
         dist.barrier()
