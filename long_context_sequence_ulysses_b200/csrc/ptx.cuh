@@ -1,5 +1,5 @@
 // ptx.cuh -- hand-written inline-PTX wrappers for sm_100a: mbarriers with
-// bounded waits, TMA tiled loads (never with cluster multicast), and the
+// bounded waits, TMA tiled loads (each CTA loads its own tiles), and the
 // tcgen05 tensor-core / tensor-memory instructions. Written from the PTX ISA
 // descriptions of these instructions.
 #pragma once
