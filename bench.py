@@ -1,11 +1,13 @@
 #!/usr/bin/env python
 """Benchmark of the Ulysses per-rank attention path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|llama8b|...] [--chunks C]
     python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
 
+By default the headline line is the llama8b workload and its "workloads"
+object holds the same measurement of tiny, long131k, million and train.
 One step = one pass of the whole hot path over the workload, for every
-emulated rank r of P:
+emulated rank r of P (rank 0 only for the million-token workload):
     seq_to_head(Q), seq_to_head(K), seq_to_head(V)   (rank r's head slice)
     attention forward (doc-bounds scan + tensor-core kernel) -> O, LSE
     [attention backward when the workload has one]
@@ -39,7 +41,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+FWD_LAUNCHES = 4   # doc-bounds (3) + the attention kernel
 BWD_LAUNCHES = 8   # doc-bounds (5) + delta, dK/dV and dQ kernels
+# Workloads the default run measures after the headline one, with the steps
+# each times (the million-token step lasts about a second: 3 are enough).
+SUB_WORKLOADS = ("tiny", "long131k", "million", "train")
+SUB_STEPS = {"million": 3}
 
 
 def load_peaks():
@@ -179,10 +186,13 @@ class Timer:
         return ((sum(xs) / len(xs)) if xs else None), (sum(xs) if xs else None)
 
 
-def build_single(U, w, inp, dev, timed):
+def build_single(U, w, inp, dev, timed, attn_ranks=None):
     """One GPU: the P ranks are emulated as P buffers, the exchanges are the
-    relayout kernels. Returns (step, our kernel launches per step, workspace)."""
+    relayout kernels. The attention runs for the ranks in ``attn_ranks``
+    (default: all of them; the million-token workload times rank 0's).
+    Returns (step, our kernel launches per step, workspace)."""
     P, N, d, Hl, Hkvl = w.P, w.N, w.d, w.Hl, w.Hkvl
+    ranks = list(range(P)) if attn_ranks is None else list(attn_ranks)
     pos = inp["position_ids"]
     q_seq, k_seq, v_seq, do_seq = inp["q"], inp["k"], inp["v"], inp.get("do")
     q_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
@@ -202,12 +212,12 @@ def build_single(U, w, inp, dev, timed):
         timed("relayout", lambda: U.seq_to_head(q_seq, P, out=q_all))
         timed("relayout", lambda: U.seq_to_head(k_seq, P, out=k_all))
         timed("relayout", lambda: U.seq_to_head(v_seq, P, out=v_all))
-        for r in range(P):
+        for r in ranks:
             timed("attn_fwd", lambda: U.attn_fwd(q_all[r], k_all[r], v_all[r], pos, out=o_all[r],
                                                  lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws))
         if w.backward:
             timed("relayout", lambda: U.seq_to_head(do_seq, P, out=do_all))
-            for r in range(P):
+            for r in ranks:
                 timed("attn_bwd", lambda: U.attn_bwd(q_all[r], k_all[r], v_all[r], o_all[r], do_all[r],
                                                      lse_all[r * Hl:(r + 1) * Hl], pos, ws=ws, dq=dq_all[r],
                                                      dk=dk_all[r], dv=dv_all[r]))
@@ -217,7 +227,7 @@ def build_single(U, w, inp, dev, timed):
         # second all-to-all: O back to sequence shards
         timed("relayout", lambda: U.head_to_seq(o_all, P, out=o_seq))
 
-    launches = 3 + 4 * P + 1 + ((1 + BWD_LAUNCHES * P + 3) if w.backward else 0)
+    launches = 3 + FWD_LAUNCHES * len(ranks) + 1 + ((1 + BWD_LAUNCHES * len(ranks) + 3) if w.backward else 0)
     return step, launches, ws
 
 
@@ -243,7 +253,7 @@ def build_fused(U, w, inp, dev):
                 U.attn_bwd_fused(q_seq, k_seq, v_seq, o_seq, do_seq, lse_all[r * Hl:(r + 1) * Hl], pos, P, r,
                                  dq=dq_seq, dk=dk_seq, dv=dv_seq, ws=ws)
 
-    return step, 4 * P + (BWD_LAUNCHES * P if w.backward else 0), ws
+    return step, FWD_LAUNCHES * P + (BWD_LAUNCHES * P if w.backward else 0), ws
 
 
 def time_fused(U, w, inp, dev, steps, total_flop):
@@ -268,10 +278,12 @@ def time_fused(U, w, inp, dev, steps, total_flop):
                     + ": sequence-sharded Q/K/V in, O out, no relayout"}
 
 
-def build_multi(U, w, inp, dev, timed, G, rank):
+def build_multi(U, w, inp, dev, timed, G, rank, chunks=1):
     """G GPUs: Ulysses with P = G real ranks. Each GPU holds tokens
     [rank*N/G, (rank+1)*N/G); the pack before and the unpack after each NCCL
-    all-to-all are the relayout kernels; each GPU computes H/G heads."""
+    all-to-all are the relayout kernels; each GPU computes H/G heads. With
+    chunks > 1 the forward takes the heads in that many chunks, the next
+    chunk's all-to-alls in flight while the current chunk is computed."""
     from long_context_sequence_ulysses_b200 import dist as udist
     N, d = w.N, w.d
     if w.H % G or w.Hkv % G or N % (G * G):
@@ -294,6 +306,17 @@ def build_multi(U, w, inp, dev, timed, G, rank):
         rdq, rdk, rdv = buf(Hg), buf(Hkvg), buf(Hkvg)
         dq_loc, dk_loc, dv_loc = torch.empty_like(q_loc), torch.empty_like(k_loc), torch.empty_like(v_loc)
 
+    if chunks > 1:
+        if w.backward:
+            raise SystemExit("--chunks applies to the forward only")
+
+        def step():
+            o, _, _, _ = timed("attn_fwd", lambda: udist.attention_forward_chunked(q_loc, k_loc, v_loc, pos_loc,
+                                                                                    chunks))
+            o_loc.copy_(o)
+
+        return step, chunks * (3 + FWD_LAUNCHES + 1), ws
+
     def step():
         udist.gather_position_ids(pos_loc, out=pos)
         q = timed("exchange", lambda: udist.seq_to_head(q_loc, send=sq, recv=rq))
@@ -308,8 +331,160 @@ def build_multi(U, w, inp, dev, timed, G, rank):
             timed("exchange", lambda: udist.head_to_seq(dv_h, recv=rdv, out=dv_loc))
         timed("exchange", lambda: udist.head_to_seq(o_head, recv=ro, out=o_loc))
 
-    launches = 3 + 4 + 1 + ((1 + BWD_LAUNCHES + 3) if w.backward else 0)
+    launches = 3 + FWD_LAUNCHES + 1 + ((1 + BWD_LAUNCHES + 3) if w.backward else 0)
     return step, launches, ws
+
+
+def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
+    """Time one workload: `warmup` untimed steps, then exactly `steps` steps
+    between a barrier and synchronisation on both sides, on the device with
+    CUDA events, clocks sampled meanwhile. Returns the JSON record of it (the
+    headline record also gets e2e, the fused step and the CPU baseline)."""
+    inp = make_inputs(w, device=dev)
+    lengths = inp["lengths"]
+    pairs, fwd_flop, bwd_flop, relayout_bytes = workload_work(w, lengths)
+    stream = torch.cuda.current_stream(dev)
+    timed = Timer(stream, False)
+    attn_ranks = [0] if w.name == "million" else None
+    if world == 1:
+        step, launches_per_step, ws = build_single(U, w, inp, dev, timed, attn_ranks)
+    else:
+        step, launches_per_step, ws = build_multi(U, w, inp, dev, timed, world, rank, args.chunks)
+        for key in ("q", "k", "v", "do"):
+            inp.pop(key, None)     # each rank keeps only its shard
+        torch.cuda.empty_cache()
+    n_attn = (1 if attn_ranks else w.P) if world == 1 else 1   # attention launches per step on this GPU
+    frac_ranks = (n_attn / w.P) if world == 1 else 1.0         # share of the attention work one step does
+    fwd_flop_step, bwd_flop_step = fwd_flop * frac_ranks, bwd_flop * frac_ranks
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    U.sync_status(ws)        # raises if a bounded device wait ran out
+    timed.enabled = args.kernel_events
+
+    sampler = ClockSampler(int(str(dev).split(":")[-1]) if ":" in str(dev) else 0)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    U.sync_status(ws)
+    ms_total = t0.elapsed_time(t1)
+    if dist is not None:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / steps
+
+    fwd_avg, fwd_sum = timed.stats("attn_fwd")
+    bwd_avg, bwd_sum = timed.stats("attn_bwd")
+    _, rel_sum = timed.stats("relayout")
+    _, exch_sum = timed.stats("exchange")
+
+    # the whole job: all ranks (all GPUs), all heads of the ranks that ran
+    total_flop = fwd_flop_step + bwd_flop_step
+    value = total_flop / (ms_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    # a kernel timed inside a step of a second or more runs at the sustained (power-capped) rate
+    long_step = ms_step > 500.0
+    bf16_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+    peak_source = "%s %s" % (peak_kind, "sustained" if long_step else "burst")
+    launches_attn = w.P * world if world == 1 else world        # attention launches over the job, all ranks
+    fwd_flop_launch = fwd_flop / launches_attn
+    bwd_flop_launch = bwd_flop / launches_attn
+    achieved = fwd_flop_launch / (fwd_avg * 1e-3) / 1e12 if fwd_avg else None
+    bwd_ach = bwd_flop_launch / (bwd_avg * 1e-3) / 1e12 if bwd_avg else None
+    traffic = lookup_traffic("attn_fwd_kernel", w.name) if world == 1 else None
+
+    def roof(kernel, ach, flop_launch, traffic_b):
+        return {"kernel": kernel, "bound": "tensor", "achieved": round(ach, 2) if ach else None, "peak": bf16_peak,
+                "peak_source": peak_source, "unit": "TFLOP/s", "frac": round(ach / bf16_peak, 4) if ach else None,
+                "frac_of_spec_2250": round(ach / SPEC_BF16_TFLOPS, 4) if ach else None, "traffic": traffic_b,
+                "flop_per_launch": flop_launch}
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "strong" if world > 1 else "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "N": w.N, "P": w.P if world == 1 else world, "H": w.H, "Hkv": w.Hkv, "d": w.d,
+            "docs": w.docs, "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
+            "step": (("seq_to_head(Q,K,V) for all P ranks; attn_fwd for "
+                      + ("rank 0's head slice" if attn_ranks else "each rank's head slice")
+                      + ("; seq_to_head(dO), attn_bwd per rank, head_to_seq(dQ,dK,dV)" if w.backward else "")
+                      + "; head_to_seq(O) for all ranks") if world == 1 else
+                     ("Ulysses over %d GPUs: pack + NCCL all-to-all of Q,K,V; attn_fwd on N x H/%d heads"
+                      % (world, world) + ("; dO exchange, attn_bwd, dQ/dK/dV exchanges" if w.backward else "")
+                      + "; O exchange + unpack"
+                      + ("; heads in %d chunks, the next chunk's exchanges in flight" % args.chunks
+                         if args.chunks > 1 else ""))),
+            "step_flop": total_flop,
+            "l2": "inputs larger than L2 (126 MB): Q alone is %d MiB" % (w.N * w.H * w.d * 2 >> 20)
+                  if w.N * w.H * w.d * 2 > (126 << 20) else
+                  "inputs smaller than L2; each step re-reads them from L2 (launch-latency bound, no roofline claim)",
+        },
+        "roofline": roof("attn_fwd_kernel (timed with the doc-bounds launch that precedes it)", achieved,
+                         fwd_flop_launch, traffic),
+        "attn_fwd_ms_per_launch": round(fwd_avg, 4) if fwd_avg else None,
+        "attn_bwd_ms_per_launch": round(bwd_avg, 4) if bwd_avg else None,
+        "attn_bwd_tflops": round(bwd_ach, 2) if bwd_ach else None,
+        "gpu_launches": launches_per_step * steps,
+        "clocks": clocks,
+    }
+    if bwd_avg:
+        out["roofline_bwd"] = roof("attn_bwd (prep, dK/dV and dQ kernels with their doc-bounds launches)", bwd_ach,
+                                   bwd_flop_launch, lookup_traffic("attn_bwd_dkdv_kernel", w.name))
+    if rel_sum:
+        rbytes = relayout_bytes
+        rb = rbytes / (rel_sum / steps * 1e-3) / 1e9
+        out["relayout"] = {"bytes_per_step": rbytes, "ms_per_step": round(rel_sum / steps, 4),
+                           "achieved_gbs": round(rb, 1), "peak_gbs": peaks["hbm_gbs"],
+                           "peak_source": peak_kind, "frac": round(rb / peaks["hbm_gbs"], 4),
+                           "frac_of_spec_8000": round(rb / SPEC_HBM_GBS, 4)}
+    if exch_sum:
+        out["exchange_ms_per_step"] = round(exch_sum / steps, 4)
+    if world > 1:
+        # device memory one step allocates beyond what is resident before it
+        # (exchange buffers and head slices; smaller with more head chunks)
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        timed.enabled = False
+        step()
+        torch.cuda.synchronize()
+        peak = torch.tensor([torch.cuda.max_memory_allocated(dev) - base], device=dev, dtype=torch.float64)
+        dist.all_reduce(peak, op=dist.ReduceOp.MAX)
+        out["step_peak_mem_bytes"] = int(peak.item())
+        out["chunks"] = args.chunks
+    if headline:
+        out["e2e"] = run_e2e(U, w, inp, args, dev) if (args.e2e_steps > 0 and world == 1) else None
+    if world == 1 and args.fused and not attn_ranks:
+        out["fused_step"] = time_fused(U, w, inp, dev, steps, total_flop)
+    if headline and rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(w, inp, args)
+    del inp, step, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_gpu(args):
@@ -326,121 +501,19 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    w = WORKLOADS[args.workload]
-    inp = make_inputs(w, device=dev)
-    lengths = inp["lengths"]
-    pairs, fwd_flop, bwd_flop, relayout_bytes = workload_work(w, lengths)
-    stream = torch.cuda.current_stream(dev)
-    timed = Timer(stream, False)
-    if world == 1:
-        step, launches_per_step, ws = build_single(U, w, inp, dev, timed)
-    else:
-        step, launches_per_step, ws = build_multi(U, w, inp, dev, timed, world, rank)
-        for key in ("q", "k", "v", "do"):
-            inp.pop(key, None)     # each rank keeps only its shard
-        torch.cuda.empty_cache()
-
-    # warm-up
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    U.sync_status(ws)        # raises if a bounded device wait ran out
-    timed.enabled = args.kernel_events
-
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    clocks = sampler.stop()
-    U.sync_status(ws)
-    ms_total = t0.elapsed_time(t1)
-    if dist is not None:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
-    ms_step = ms_total / args.steps
-
-    fwd_avg, _ = timed.stats("attn_fwd")
-    bwd_avg, _ = timed.stats("attn_bwd")
-    _, rel_sum = timed.stats("relayout")
-    _, exch_sum = timed.stats("exchange")
-
-    total_flop = fwd_flop + bwd_flop          # the whole job (all ranks, all heads)
-    value = total_flop / (ms_step * 1e-3) / 1e12
-    peaks, peak_kind = load_peaks()
-    long_step = ms_total > 1000.0
-    bf16_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
-    launches_attn_fwd = (w.P if world == 1 else 1) * world    # attention launches per step over the job
-    fwd_flop_launch = fwd_flop / launches_attn_fwd
-    achieved = fwd_flop_launch / (fwd_avg * 1e-3) / 1e12 if fwd_avg else None
-    traffic = lookup_traffic("attn_fwd_kernel", w.name) if world == 1 else None
-    e2e = run_e2e(U, w, inp, args, dev) if (args.e2e_steps > 0 and world == 1) else None
-
-    out = {
-        "metric": METRIC,
-        "value": round(value, 2),
-        "unit": "TFLOP/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True,
-        "scaling": "strong" if world > 1 else "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic",
-        "config": {
-            "workload": w.name, "N": w.N, "P": w.P if world == 1 else world, "H": w.H, "Hkv": w.Hkv, "d": w.d,
-            "docs": w.docs, "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
-            "step": (("seq_to_head(Q,K,V) for all P ranks; attn_fwd for each rank's head slice"
-                      + ("; seq_to_head(dO), attn_bwd per rank, head_to_seq(dQ,dK,dV)" if w.backward else "")
-                      + "; head_to_seq(O) for all ranks") if world == 1 else
-                     ("Ulysses over %d GPUs: pack + NCCL all-to-all of Q,K,V; attn_fwd on N x H/%d heads"
-                      % (world, world) + ("; dO exchange, attn_bwd, dQ/dK/dV exchanges" if w.backward else "")
-                      + "; O exchange + unpack")),
-            "l2": "inputs larger than L2 (126 MB): Q alone is %d MiB" % (w.N * w.H * w.d * 2 >> 20),
-        },
-        "roofline": {
-            "kernel": "attn_fwd_kernel (timed with the doc-bounds scan it is launched with)",
-            "bound": "tensor",
-            "achieved": round(achieved, 2) if achieved else None,
-            "peak": bf16_peak,
-            "peak_source": ("%s %s" % (peak_kind, "sustained" if long_step else "burst")),
-            "unit": "TFLOP/s",
-            "frac": round(achieved / bf16_peak, 4) if achieved else None,
-            "frac_of_spec_2250": round(achieved / SPEC_BF16_TFLOPS, 4) if achieved else None,
-            "traffic": traffic,
-            "flop_per_launch": fwd_flop_launch,
-        },
-        "attn_fwd_ms_per_launch": round(fwd_avg, 4) if fwd_avg else None,
-        "attn_bwd_ms_per_launch": round(bwd_avg, 4) if bwd_avg else None,
-        "attn_bwd_tflops": round((bwd_flop / launches_attn_fwd) / (bwd_avg * 1e-3) / 1e12, 2) if bwd_avg else None,
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks,
-        "e2e": e2e,
-    }
-    if rel_sum:
-        rb = relayout_bytes / (rel_sum / args.steps * 1e-3) / 1e9
-        out["relayout"] = {"bytes_per_step": relayout_bytes, "ms_per_step": round(rel_sum / args.steps, 4),
-                           "achieved_gbs": round(rb, 1), "peak_gbs": peaks["hbm_gbs"],
-                           "frac": round(rb / peaks["hbm_gbs"], 4), "frac_of_spec_8000": round(rb / SPEC_HBM_GBS, 4)}
-    if exch_sum:
-        out["exchange_ms_per_step"] = round(exch_sum / args.steps, 4)
-    if world == 1 and args.fused:
-        out["fused_step"] = time_fused(U, w, inp, dev, args.steps, total_flop)
-    if rank == 0 and not args.no_cpu_baseline and world == 1:
-        out["cpu_baseline"] = cpu_baseline(w, inp, args)
+    name = "llama8b" if args.workload == "all" else args.workload
+    out = measure(U, WORKLOADS[name], dev, args, args.steps, args.warmup, world, rank, dist, headline=True)
+    if args.workload == "all" and world == 1:
+        subs = {}
+        for sub in SUB_WORKLOADS:
+            k = SUB_STEPS.get(sub, args.steps)
+            r = measure(U, WORKLOADS[sub], dev, args, k, max(3, args.warmup if sub != "million" else 3), world,
+                        rank, dist, headline=False)
+            for key in ("metric", "unit", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "dtype", "data"):
+                r.pop(key, None)
+            subs[sub] = r
+        out["workloads"] = subs
+        out["gpu_launches"] += sum(r["gpu_launches"] for r in subs.values())
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -538,56 +611,79 @@ def _oracle_rows_sample(w, lengths, budget_pairs: float, seed: int):
     return rows, int(keys[rows].sum()) * w.Hl
 
 
-def cpu_baseline(w, inp, args, seconds_target: float = 15.0):
-    """The fp64 oracle timed on this host's cores on a bounded sample of rank
-    0's rows; its rate is scaled to TFLOP/s with the same FLOP count per pair."""
-    import numpy as np
-    import oracle
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+def _oracle_slice(w, inp):
     q = inp["q"][:, :w.Hl].contiguous().cpu()
     k = inp["k"][:, :w.Hkvl].contiguous().cpu()
     v = inp["v"][:, :w.Hkvl].contiguous().cpu()
-    pos = inp["position_ids"].cpu()
-    # calibrate on a small sample, then size the timed sample to ~seconds_target
+    return q, k, v, inp["position_ids"].cpu()
+
+
+def _oracle_rate(w, inp, sl):
+    """Query-key pairs per second of the oracle on a small calibration sample."""
+    import oracle
     rows, pr = _oracle_rows_sample(w, inp["lengths"], 2e6, seed=1)
     t = time.perf_counter()
-    oracle.attn_fwd(q, k, v, pos, rows=rows)
-    dt = max(time.perf_counter() - t, 1e-3)
-    rate = pr / dt
-    rows, pr = _oracle_rows_sample(w, inp["lengths"], rate * seconds_target, seed=2)
+    oracle.attn_fwd(*sl, rows=rows)
+    return pr / max(time.perf_counter() - t, 1e-3)
+
+
+def _oracle_step(w, inp, sl, rate, seconds_target, seed):
+    """One timed oracle run on about seconds_target of rank 0's rows.
+    Returns (seconds, pairs, rows)."""
+    import oracle
+    rows, pr = _oracle_rows_sample(w, inp["lengths"], rate * seconds_target, seed=seed)
     t = time.perf_counter()
-    oracle.attn_fwd(q, k, v, pos, rows=rows)
-    dt = time.perf_counter() - t
+    oracle.attn_fwd(*sl, rows=rows)
+    return time.perf_counter() - t, pr, len(rows)
+
+
+def cpu_baseline(w, inp, args, seconds_target: float = 15.0):
+    """The fp64 oracle timed on this host's cores on a bounded sample of rank
+    0's rows; its rate is scaled to TFLOP/s with the same FLOP count per pair."""
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sl = _oracle_slice(w, inp)
+    dt, pr, nrows = _oracle_step(w, inp, sl, _oracle_rate(w, inp, sl), seconds_target, seed=2)
     flop = 4.0 * w.d * pr
     return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": "forward attention of %d rows x %d heads of rank 0 (%d query-key pairs, %.1f s)"
-                      % (len(rows), w.Hl, pr, dt)}
+                      % (nrows, w.Hl, pr, dt)}
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, on this host's cores.
+    Each step is a bounded sample of rank 0's rows of the workload (about
+    --ref-seconds of work); value and ms_per_step are those of the sampled work
+    actually timed, not an extrapolation to the whole step."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = WORKLOADS["llama8b" if args.workload == "all" else args.workload]
     inp = make_inputs(w, device="cpu")
-    steps = []
-    base = None
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sl = _oracle_slice(w, inp)
+    rate = _oracle_rate(w, inp, sl)
+    times, pairs = [], []
     for i in range(args.warmup + args.steps):
-        base = cpu_baseline(w, inp, args, seconds_target=args.ref_seconds)
+        dt, pr, nrows = _oracle_step(w, inp, sl, rate, args.ref_seconds, seed=2 + i)
         if i >= args.warmup:
-            steps.append(base["value"])
-    value = sum(steps) / len(steps)
-    pairs, fwd_flop, bwd_flop, _ = workload_work(w, inp["lengths"])
-    ms_step = (fwd_flop + bwd_flop) / (value * 1e12) * 1e3
+            times.append(dt)
+            pairs.append(pr)
+    flop = 4.0 * w.d * sum(pairs)
+    value = flop / sum(times) / 1e12
+    ms_step = sum(times) / len(times) * 1e3
     out = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "N": w.N, "P": w.P, "H": w.H, "Hkv": w.Hkv, "d": w.d, "docs": w.docs,
-                   "note": "each step times the fp64 CPU oracle on a bounded sample of rank 0's rows; "
-                           "ms_per_step is the extrapolated time of the whole step"},
-        "cpu_baseline": dict(base, value=round(value, 6)),
+                   "note": "each step times the fp64 CPU oracle on a bounded sample of rank 0's rows (about "
+                           "%.0f s of host work, %d query-key pairs on average); value and ms_per_step are "
+                           "those of the sampled work" % (args.ref_seconds, sum(pairs) // len(pairs))},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": "forward attention of rank 0's rows x %d heads, %d steps of about %.0f s "
+                                   "(%d query-key pairs in all)" % (w.Hl, len(times), args.ref_seconds,
+                                                                     sum(pairs))},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
@@ -598,14 +694,19 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="llama8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(WORKLOADS),
+                    help="all (default): llama8b as the headline line, the other workloads in its 'workloads' "
+                         "object; or one workload alone")
+    ap.add_argument("--chunks", type=int, default=1,
+                    help="multi-GPU forward with the heads in this many chunks (head-chunked Ulysses)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fused", dest="fused", action="store_false",
                     help="skip the extra timing of the step with the exchanges fused into the attention")
     ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
-    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=4.0,
+                    help="host seconds of oracle work per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "b200":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

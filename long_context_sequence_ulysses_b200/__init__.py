@@ -99,16 +99,50 @@ def _stream(t: torch.Tensor):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
-def _bf16_cuda(name: str, t: torch.Tensor, ndim: int) -> None:
-    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA bf16 tensor")
-    if t.dim() != ndim or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor, got shape {tuple(t.shape)}")
+def _spec(name: str, t, shape, dtype=torch.bfloat16) -> None:
+    """Shape, dtype and contiguity of a buffer the C call reads or writes.
+
+    The C ABI derives every size from N, the head counts and d, so a buffer
+    smaller than that would be read or written past its end: every tensor is
+    checked against the exact shape the call implies. Raised as ValueError
+    (TypeError if it is not a tensor); the device is checked separately."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _same_cuda(*named) -> None:
+    """Every tensor on one CUDA device."""
+    dev = None
+    for name, t in named:
+        if not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+
+
+def _dims(name: str, t, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    return tuple(t.shape)
 
 
 def _pos32(pos: torch.Tensor, N: int) -> torch.Tensor:
-    if pos.dim() != 1 or pos.shape[0] != N or not pos.is_cuda:
-        raise ValueError("position_ids must be a 1-D CUDA tensor of length N")
+    if not isinstance(pos, torch.Tensor) or pos.dim() != 1 or pos.shape[0] != N:
+        raise ValueError("position_ids must be a 1-D tensor of length N")
+    if pos.dtype not in (torch.int32, torch.int64):
+        raise ValueError("position_ids must be int32 or int64")
+    if not pos.is_cuda:
+        raise TypeError("position_ids must be a CUDA tensor")
     if pos.dtype != torch.int32:
         pos = pos.to(torch.int32)   # argument marshalling: the ABI takes int32 ids
     return pos.contiguous()
@@ -117,13 +151,17 @@ def _pos32(pos: torch.Tensor, N: int) -> torch.Tensor:
 def seq_to_head(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """[N][Hx][d] (= P rank buffers [P][N/P][Hx][d]) -> [P][N][Hx/P][d], or
     rank r's slice [N][Hx/P][d] when ``rank >= 0``."""
-    _bf16_cuda("src", src, 3)
-    N, Hx, d = src.shape
+    N, Hx, d = _dims("src", src, 3)
+    _spec("src", src, (N, Hx, d))
+    if P < 1 or Hx % P:
+        raise ValueError(f"head count {Hx} must be divisible by P={P}")
     shape = (P, N, Hx // P, d) if rank < 0 else (N, Hx // P, d)
-    if out is None:
+    if out is not None:
+        _spec("out", out, shape)
+        _same_cuda(("src", src), ("out", out))
+    else:
+        _same_cuda(("src", src))
         out = torch.empty(shape, dtype=src.dtype, device=src.device)
-    elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != src.dtype:
-        raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
     _check(_lib.ulysses_seq_to_head(_ptr(src), _ptr(out), N, P, Hx, d, rank, _stream(src)))
     return out
 
@@ -132,21 +170,23 @@ def head_to_seq(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.T
     """[P][N][Hx/P][d] -> [N][Hx][d]; with ``rank >= 0`` src is rank r's slice
     [N][Hx/P][d] and only its heads of ``out`` are written."""
     if rank < 0:
-        _bf16_cuda("src", src, 4)
-        Pp, N, Hl, d = src.shape
+        Pp, N, Hl, d = _dims("src", src, 4)
         if Pp != P:
             raise ValueError("src.shape[0] must equal P")
+        _spec("src", src, (P, N, Hl, d))
     else:
-        _bf16_cuda("src", src, 3)
-        N, Hl, d = src.shape
+        N, Hl, d = _dims("src", src, 3)
+        _spec("src", src, (N, Hl, d))
     Hx = Hl * P
     shape = (N, Hx, d)
-    if out is None:
+    if out is not None:
+        _spec("out", out, shape)
+        _same_cuda(("src", src), ("out", out))
+    else:
         if rank >= 0:
             raise ValueError("head_to_seq with rank >= 0 needs `out` (other ranks' heads are kept)")
+        _same_cuda(("src", src))
         out = torch.empty(shape, dtype=src.dtype, device=src.device)
-    elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != src.dtype:
-        raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
     _check(_lib.ulysses_head_to_seq(_ptr(src), _ptr(out), N, P, Hx, d, rank, _stream(src)))
     return out
 
@@ -156,9 +196,21 @@ def workspace_bytes(N: int, Hl: int, Hkvl: int, d: int, backward: bool = False) 
 
 
 def _workspace(ws: Optional[torch.Tensor], nbytes: int, device) -> torch.Tensor:
-    if ws is None or ws.numel() * ws.element_size() < nbytes:
-        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
-    return ws
+    """The caller's workspace if it is a large enough uint8 buffer on the
+    device, else a fresh one."""
+    if ws is not None:
+        if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or not ws.is_contiguous():
+            raise ValueError("ws must be a contiguous uint8 tensor")
+        if ws.device != device:
+            raise ValueError(f"ws is on {ws.device}, expected {device}")
+        if ws.numel() >= nbytes:
+            return ws
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _heads_ok(Hl: int, Hkvl: int) -> None:
+    if Hl < 1 or Hkvl < 1 or Hl % Hkvl:
+        raise ValueError(f"query heads ({Hl}) must be a positive multiple of KV heads ({Hkvl})")
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position_ids: torch.Tensor,
@@ -169,12 +221,20 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position_ids: to
 
     q [N][Hl][d], k/v [N][Hkvl][d] bf16; position_ids [N]. Returns
     (o [N][Hl][d] bf16, lse [Hl][N] fp32)."""
-    _bf16_cuda("q", q, 3); _bf16_cuda("k", k, 3); _bf16_cuda("v", v, 3)
-    N, Hl, d = q.shape
-    Hkvl = k.shape[1]
-    if k.shape != (N, Hkvl, d) or v.shape != k.shape:
-        raise ValueError("k and v must be [N][Hkvl][d]")
+    N, Hl, d = _dims("q", q, 3)
+    Hkvl = _dims("k", k, 3)[1]
+    _spec("q", q, (N, Hl, d))
+    _spec("k", k, (N, Hkvl, d))
+    _spec("v", v, (N, Hkvl, d))
+    _heads_ok(Hl, Hkvl)
+    if out is not None:
+        _spec("out", out, (N, Hl, d))
+    if lse is not None:
+        _spec("lse", lse, (Hl, N), torch.float32)
     pos = _pos32(position_ids, N)
+    _same_cuda(("q", q), ("k", k), ("v", v), *((("out", out),) if out is not None else ()),
+               *((("lse", lse),) if lse is not None else ()))
+    _same_cuda(("q", q), ("position_ids", pos))
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
@@ -187,6 +247,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position_ids: to
     return out, lse
 
 
+def _rank_heads(H: int, Hkv: int, P: int, rank: int) -> Tuple[int, int]:
+    if P < 1 or H % P or Hkv % P:
+        raise ValueError(f"H={H} and Hkv={Hkv} must be divisible by P={P}")
+    if not 0 <= rank < P:
+        raise ValueError(f"rank={rank} outside [0, {P})")
+    _heads_ok(H // P, Hkv // P)
+    return H // P, Hkv // P
+
+
 def attn_fwd_fused(q_seq: torch.Tensor, k_seq: torch.Tensor, v_seq: torch.Tensor, position_ids: torch.Tensor,
                    P: int, rank: int, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                    lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
@@ -194,16 +263,25 @@ def attn_fwd_fused(q_seq: torch.Tensor, k_seq: torch.Tensor, v_seq: torch.Tensor
     """Attention of rank ``rank``'s heads read straight from the
     sequence-sharded buffers q_seq [N][H][d], k_seq/v_seq [N][Hkv][d]; O is
     written into ``out`` [N][H][d] (only this rank's heads)."""
-    _bf16_cuda("q_seq", q_seq, 3); _bf16_cuda("k_seq", k_seq, 3); _bf16_cuda("v_seq", v_seq, 3)
-    N, H, d = q_seq.shape
-    Hkv = k_seq.shape[1]
+    N, H, d = _dims("q_seq", q_seq, 3)
+    Hkv = _dims("k_seq", k_seq, 3)[1]
+    _spec("q_seq", q_seq, (N, H, d))
+    _spec("k_seq", k_seq, (N, Hkv, d))
+    _spec("v_seq", v_seq, (N, Hkv, d))
+    Hl, Hkvl = _rank_heads(H, Hkv, P, rank)
+    if out is not None:
+        _spec("out", out, (N, H, d))
+    if lse is not None:
+        _spec("lse", lse, (Hl, N), torch.float32)
     pos = _pos32(position_ids, N)
+    _same_cuda(("q_seq", q_seq), ("k_seq", k_seq), ("v_seq", v_seq),
+               *((("out", out),) if out is not None else ()), *((("lse", lse),) if lse is not None else ()))
+    _same_cuda(("q_seq", q_seq), ("position_ids", pos))
     if out is None:
         out = torch.empty_like(q_seq)
-    Hl, Hkvl = H // P, Hkv // P
     if lse is None:
-        lse = torch.empty((max(Hl, 1), N), dtype=torch.float32, device=q_seq.device)
-    nbytes = workspace_bytes(N, max(Hl, 1), max(Hkvl, 1), d, False)
+        lse = torch.empty((Hl, N), dtype=torch.float32, device=q_seq.device)
+    nbytes = workspace_bytes(N, Hl, Hkvl, d, False)
     ws = _workspace(ws, nbytes, q_seq.device)
     sc = 0.0 if scale is None else float(scale)
     _check(_lib.ulysses_attn_fwd_fused(_ptr(q_seq), _ptr(k_seq), _ptr(v_seq), _ptr(pos), N, P, H, Hkv, d, rank,
@@ -217,13 +295,22 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, dk, dv) of sum(dout * o) for one rank's head slice."""
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
-        _bf16_cuda(name, t, 3)
-    N, Hl, d = q.shape
-    Hkvl = k.shape[1]
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (Hl, N) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [Hl][N] tensor")
+    N, Hl, d = _dims("q", q, 3)
+    Hkvl = _dims("k", k, 3)[1]
+    qshape, kshape = (N, Hl, d), (N, Hkvl, d)
+    for name, t, shp in (("q", q, qshape), ("k", k, kshape), ("v", v, kshape), ("o", o, qshape),
+                         ("dout", dout, qshape)):
+        _spec(name, t, shp)
+    _spec("lse", lse, (Hl, N), torch.float32)
+    _heads_ok(Hl, Hkvl)
+    named = [("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("lse", lse)]
+    for name, t, shp in (("dq", dq, qshape), ("dk", dk, kshape), ("dv", dv, kshape)):
+        if t is not None:
+            _spec(name, t, shp)
+            named.append((name, t))
     pos = _pos32(position_ids, N)
+    _same_cuda(*named)
+    _same_cuda(("q", q), ("position_ids", pos))
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -262,18 +349,27 @@ def attn_bwd_fused(q_seq: torch.Tensor, k_seq: torch.Tensor, v_seq: torch.Tensor
     """Gradients of rank ``rank``'s heads read straight from the sequence-sharded
     buffers (q/o/dout [N][H][d], k/v [N][Hkv][d]) and written into dq [N][H][d],
     dk / dv [N][Hkv][d] (only this rank's heads); lse is [H/P][N]."""
-    for name, t in (("q_seq", q_seq), ("k_seq", k_seq), ("v_seq", v_seq), ("o_seq", o_seq), ("dout_seq", dout_seq)):
-        _bf16_cuda(name, t, 3)
-    N, H, d = q_seq.shape
-    Hkv = k_seq.shape[1]
-    Hl, Hkvl = H // P, Hkv // P
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (Hl, N) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [H/P][N] tensor")
+    N, H, d = _dims("q_seq", q_seq, 3)
+    Hkv = _dims("k_seq", k_seq, 3)[1]
+    qshape, kshape = (N, H, d), (N, Hkv, d)
+    for name, t, shp in (("q_seq", q_seq, qshape), ("k_seq", k_seq, kshape), ("v_seq", v_seq, kshape),
+                         ("o_seq", o_seq, qshape), ("dout_seq", dout_seq, qshape)):
+        _spec(name, t, shp)
+    Hl, Hkvl = _rank_heads(H, Hkv, P, rank)
+    _spec("lse", lse, (Hl, N), torch.float32)
+    named = [("q_seq", q_seq), ("k_seq", k_seq), ("v_seq", v_seq), ("o_seq", o_seq), ("dout_seq", dout_seq),
+             ("lse", lse)]
+    for name, t, shp in (("dq", dq, qshape), ("dk", dk, kshape), ("dv", dv, kshape)):
+        if t is not None:
+            _spec(name, t, shp)
+            named.append((name, t))
     pos = _pos32(position_ids, N)
+    _same_cuda(*named)
+    _same_cuda(("q_seq", q_seq), ("position_ids", pos))
     dq = torch.empty_like(q_seq) if dq is None else dq
     dk = torch.empty_like(k_seq) if dk is None else dk
     dv = torch.empty_like(v_seq) if dv is None else dv
-    nbytes = workspace_bytes(N, max(Hl, 1), max(Hkvl, 1), d, True)
+    nbytes = workspace_bytes(N, Hl, Hkvl, d, True)
     ws = _workspace(ws, nbytes, q_seq.device)
     sc = 0.0 if scale is None else float(scale)
     _check(_lib.ulysses_attn_bwd_fused(_ptr(q_seq), _ptr(k_seq), _ptr(v_seq), _ptr(o_seq), _ptr(dout_seq), _ptr(lse),

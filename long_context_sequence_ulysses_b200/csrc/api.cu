@@ -61,6 +61,8 @@ EncodeTiledFn encode_fn()
 
 int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
 
+void clear_last_error() { g_err[0] = 0; }
+
 int num_sms_current_device()
 {
     static int cache[64] = {};
@@ -156,6 +158,13 @@ static int check_attn_shapes(const char *name, int64_t N, int Hl, int Hkvl, int 
     if (Hl < 1 || Hkvl < 1) return fail(ULYSSES_ERR_INVALID, "%s: head counts must be >= 1", name);
     if (Hl % Hkvl) return fail(ULYSSES_ERR_INVALID, "%s: Hl=%d not divisible by Hkvl=%d", name, Hl, Hkvl);
     if (!head_dim_ok(d)) return fail(ULYSSES_ERR_INVALID, "%s: d=%d not in {32,64,128}", name, d);
+    // Work items, CTA counts and the backward's per-row launch are 32-bit: at
+    // most Hl * ceil(N/128) * 16 of them (the backward's per-row grid, the
+    // largest) may be launched.
+    const int64_t T = (N + kTileM - 1) / kTileM;
+    if (int64_t(Hl) * T * 16 > INT32_MAX)
+        return fail(ULYSSES_ERR_UNSUPPORTED, "%s: Hl * ceil(N/128) = %lld exceeds the 32-bit launch limit of %d",
+                    name, (long long)(int64_t(Hl) * T), INT32_MAX / 16);
     return ULYSSES_OK;
 }
 

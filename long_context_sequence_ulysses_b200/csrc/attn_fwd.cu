@@ -675,7 +675,8 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.status = reinterpret_cast<uint32_t *>(const_cast<char *>(a.ws) + a.L.status);
     p.pair_heads = fwd_pairs_heads(a.Hl, a.Hkvl) ? 1 : 0;
     const int64_t items = p.pair_heads ? int64_t(p.T) * (a.Hl / 2) : ceil_div(p.T, 2) * a.Hl;
-    if (items > INT32_MAX) return cudaErrorInvalidValue;   // the work counter and item indices are 32-bit
+    // the work counter and item indices are 32-bit; check_attn_shapes rejects larger problems
+    if (items > INT32_MAX) return cudaErrorInvalidValue;
     p.items = static_cast<int>(items);
     p.wait_limit_ns = a.wait_limit_ns;
     p.debug_flags = a.debug_flags;

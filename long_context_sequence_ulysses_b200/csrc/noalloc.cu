@@ -73,6 +73,7 @@ extern "C" int ulysses_attn_fwd_noalloc(const void *q, const void *k, const void
                                         void *stream)
 {
     using namespace uly;
+    clear_last_error();
     if (N > kNoAllocMaxTokens)
         return set_last_error(ULYSSES_ERR_UNSUPPORTED,
                               "ulysses_attn_fwd_noalloc: N exceeds the static scratch limit of 131072 tokens");

@@ -112,6 +112,7 @@ cudaError_t launch_attn_bwd(const BwdLaunch &a, cudaStream_t stream);
 // api.cu
 int num_sms_current_device();
 int set_last_error(int code, const char *msg);   // records msg for ulysses_last_error(); returns code
+void clear_last_error();
 bool encode_tmap_3d(void *tmap /*CUtensorMap*/, const void *base, int64_t inner, int64_t mid, int64_t outer,
                     int64_t mid_stride_bytes, int64_t outer_stride_bytes, int box_inner, int box_outer,
                     int swizzle_bytes);

@@ -91,9 +91,11 @@ def gather_position_ids(pos_local: torch.Tensor, group=None, out: Optional[torch
 
 def attention_forward(q_local: torch.Tensor, k_local: torch.Tensor, v_local: torch.Tensor,
                       pos_local: torch.Tensor, group=None, scale: Optional[float] = None,
-                      attn: Optional[Callable] = None, pack=None, unpack=None):
+                      attn: Optional[Callable] = None, pack=None, unpack=None, keep_for_backward: bool = False):
     """The Ulysses attention step of one rank: returns (o_local [N/G][H][d],
-    lse [H/G][N] for this rank's heads, position ids of the whole sequence)."""
+    lse [H/G][N] for this rank's heads, position ids of the whole sequence).
+    With ``keep_for_backward`` a fourth item holds what the backward needs:
+    this rank's head slices (q, k, v, o), each [N][heads/G][d]."""
     pos = gather_position_ids(pos_local, group)
     q = seq_to_head(q_local, group, pack)
     k = seq_to_head(k_local, group, pack)
@@ -102,7 +104,30 @@ def attention_forward(q_local: torch.Tensor, k_local: torch.Tensor, v_local: tor
         import long_context_sequence_ulysses_b200 as U
         attn = U.attn_fwd
     o, lse = attn(q, k, v, pos, scale=scale)
-    return head_to_seq(o, group, unpack), lse, pos
+    o_local = head_to_seq(o, group, unpack)
+    if keep_for_backward:
+        return o_local, lse, pos, (q, k, v, o)
+    return o_local, lse, pos
+
+
+def attention_backward(saved, lse: torch.Tensor, pos: torch.Tensor, dout_local: torch.Tensor, group=None,
+                       scale: Optional[float] = None, attn_bwd: Optional[Callable] = None, pack=None,
+                       unpack=None):
+    """The backward of the Ulysses attention step of one rank. The upstream
+    gradient arrives sequence-sharded like O, so it crosses the first exchange
+    (dO [N/G][H][d] -> [N][H/G][d]); the gradients of this rank's heads are
+    computed locally, as in the forward (heads are independent); dQ, dK and dV
+    cross the second exchange back to sequence shards. ``saved`` is the
+    (q, k, v, o) head slices attention_forward keeps; lse and pos are its
+    other outputs. Returns (dq_local [N/G][H][d], dk_local, dv_local
+    [N/G][Hkv][d])."""
+    q, k, v, o = saved
+    g = seq_to_head(dout_local, group, pack)
+    if attn_bwd is None:
+        import long_context_sequence_ulysses_b200 as U
+        attn_bwd = U.attn_bwd
+    dq, dk, dv = attn_bwd(q, k, v, o, g, lse, pos, scale=scale)
+    return head_to_seq(dq, group, unpack), head_to_seq(dk, group, unpack), head_to_seq(dv, group, unpack)
 
 
 def attention_forward_chunked(q_local: torch.Tensor, k_local: torch.Tensor, v_local: torch.Tensor,

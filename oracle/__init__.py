@@ -12,6 +12,7 @@ Parity status of each function (what pins it is listed in the tests):
   doc_start                 pinned (hand-derived golden, definition by brute force)
   attn_fwd                  pinned (brute force, SDPA, closed forms, invariances)
   attn_bwd                  pinned (finite differences, autograd, sum rules)
+  attn_bwd_sampled          pinned (equal to attn_bwd on the sampled rows and keys)
 """
 from __future__ import annotations
 
@@ -58,6 +59,8 @@ def _load():
             lib.oracle_attn_fwd_rows.restype = I32
             lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, I64, I32, I32, I32, F64, P, P, P, P, P]
             lib.oracle_attn_bwd.restype = I32
+            lib.oracle_attn_bwd_sampled.argtypes = [P, P, P, P, P, I64, I32, I32, I32, F64, P, I64, P, I64, P, P, P]
+            lib.oracle_attn_bwd_sampled.restype = I32
             _lib = lib
     return _lib
 
@@ -161,3 +164,26 @@ def attn_bwd(q, k, v, dout, pos, scale: Optional[float] = None):
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd failed ({rc})")
     return dq, dk, dv, o, lse
+
+
+def attn_bwd_sampled(q, k, v, dout, pos, rows: Sequence[int], keys: Sequence[int], scale: Optional[float] = None):
+    """The exact gradients of sum(dO * O) only where asked: dq [len(rows)][Hl][d]
+    for the query rows ``rows`` and dk, dv [len(keys)][Hkvl][d] for the keys
+    ``keys``, in fp64 (same formulas as attn_bwd)."""
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    N, Hl, d = qb.shape
+    Hkvl = kb.shape[1]
+    p = _i32(pos)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    kk = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
+    dq = np.empty((r.shape[0], Hl, d), dtype=np.float64)
+    dk = np.empty((kk.shape[0], Hkvl, d), dtype=np.float64)
+    dv = np.empty((kk.shape[0], Hkvl, d), dtype=np.float64)
+    rc = _load().oracle_attn_bwd_sampled(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(p), N, Hl, Hkvl, d,
+                                         float(scale), _ptr(r), r.shape[0], _ptr(kk), kk.shape[0], _ptr(dq),
+                                         _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd_sampled failed ({rc})")
+    return dq, dk, dv

@@ -285,3 +285,136 @@ done:
     free(ds); free(de); free(O); free(LSE); free(D);
     return err;
 }
+
+/* ------------------------------------------------------------------------ */
+/* attention backward on sampled rows and keys                              */
+/* ------------------------------------------------------------------------ */
+
+/* The same gradients as oracle_attn_bwd, evaluated only where asked: dQ for
+ * the query rows rows[0..nrows) and dK, dV for the keys keys[0..nkeys). This
+ * lets a long document's heaviest keys (its first ones, which every later
+ * query of the document attends to) be checked without the whole backward.
+ * Every query row whose values enter those results (the sampled rows, and
+ * rows j .. end of document - 1 of every sampled key j) first gets its exact
+ * forward values (LSE_i, and D_i = sum_c dO_ic O_ic); then
+ *   dQ_i = scale * sum_{j in [doc_start(i), i]} dS_ij k_j
+ *   dK_j = scale * sum_{h in group} sum_{i in [j, doc end)} dS_ij q_i
+ *   dV_j = sum_{h in group} sum_{i in [j, doc end)} P_ij dO_i
+ * with P_ij = exp(scale q_i.k_j - LSE_i) and dS_ij = P_ij (dO_i.v_j - D_i).
+ * Outputs: dq [nrows][Hl][d], dk and dv [nkeys][Hkvl][d], fp64.            */
+int oracle_attn_bwd_sampled(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *dout, const int32_t *pos, int64_t N, int Hl,
+                            int Hkvl, int d, double scale, const int64_t *rows, int64_t nrows,
+                            const int64_t *keys, int64_t nkeys, double *dq, double *dk, double *dv)
+{
+    if (Hkvl <= 0 || Hl % Hkvl != 0) return -1;
+    const int G = Hl / Hkvl;
+    const size_t nz = (size_t)(N > 0 ? N : 1);
+    int32_t *ds = (int32_t *)malloc(sizeof(int32_t) * nz);
+    int64_t *de = (int64_t *)malloc(sizeof(int64_t) * nz);
+    unsigned char *need = (unsigned char *)calloc(nz, 1);
+    double *LSE = (double *)malloc(sizeof(double) * nz * Hl);
+    double *D = (double *)malloc(sizeof(double) * nz * Hl);
+    if (!ds || !de || !need || !LSE || !D) {
+        free(ds); free(de); free(need); free(LSE); free(D);
+        return -2;
+    }
+    oracle_doc_start(pos, N, ds);
+    for (int64_t i = N - 1, end = N; i >= 0; --i) {
+        de[i] = end;
+        if (ds[i] == i) end = i;
+    }
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (rows[r] < 0 || rows[r] >= N) { free(ds); free(de); free(need); free(LSE); free(D); return -1; }
+        need[rows[r]] = 1;
+    }
+    for (int64_t t = 0; t < nkeys; ++t) {
+        if (keys[t] < 0 || keys[t] >= N) { free(ds); free(de); free(need); free(LSE); free(D); return -1; }
+        for (int64_t i = keys[t]; i < de[keys[t]]; ++i) need[i] = 1;
+    }
+    int err = 0;
+
+    /* Step 1: forward values and D_i of every row that is needed. */
+    #pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * nz);
+        double *oi = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!s_buf || !oi) {
+            #pragma omp atomic write
+            err = -2;
+        } else {
+            #pragma omp for collapse(2) schedule(dynamic, 4)
+            for (int h = 0; h < Hl; ++h)
+                for (int64_t i = 0; i < N; ++i) {
+                    if (!need[i]) continue;
+                    attn_row(q, k, v, i, ds[i], h, h / G, Hl, Hkvl, d, scale, s_buf, oi,
+                             LSE + (int64_t)h * N + i);
+                    const uint16_t *gi = dout + (i * Hl + h) * (int64_t)d;
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c) acc += bf16_to_f64(gi[c]) * oi[c];
+                    D[(int64_t)h * N + i] = acc;
+                }
+        }
+        free(s_buf);
+        free(oi);
+    }
+    if (err) goto done;
+
+    /* Step 2: dQ of the sampled rows. */
+    #pragma omp parallel for collapse(2) schedule(dynamic, 4)
+    for (int h = 0; h < Hl; ++h)
+        for (int64_t r = 0; r < nrows; ++r) {
+            const int64_t i = rows[r];
+            const int kvh = h / G;
+            const uint16_t *qi = q + (i * Hl + h) * (int64_t)d;
+            const uint16_t *gi = dout + (i * Hl + h) * (int64_t)d;
+            double *dqi = dq + (r * Hl + h) * (int64_t)d;
+            for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+            for (int64_t j = ds[i]; j <= i; ++j) {
+                const uint16_t *kj = k + (j * Hkvl + kvh) * (int64_t)d;
+                const uint16_t *vj = v + (j * Hkvl + kvh) * (int64_t)d;
+                double s = 0.0, dp = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    s += bf16_to_f64(qi[c]) * bf16_to_f64(kj[c]);
+                    dp += bf16_to_f64(gi[c]) * bf16_to_f64(vj[c]);
+                }
+                const double p = exp(scale * s - LSE[(int64_t)h * N + i]);
+                const double dsij = p * (dp - D[(int64_t)h * N + i]);
+                for (int c = 0; c < d; ++c) dqi[c] += scale * dsij * bf16_to_f64(kj[c]);
+            }
+        }
+
+    /* Step 3: dK and dV of the sampled keys, summed over the group's query heads. */
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int kvh = 0; kvh < Hkvl; ++kvh)
+        for (int64_t t = 0; t < nkeys; ++t) {
+            const int64_t j = keys[t];
+            const uint16_t *kj = k + (j * Hkvl + kvh) * (int64_t)d;
+            const uint16_t *vj = v + (j * Hkvl + kvh) * (int64_t)d;
+            double *dkj = dk + (t * Hkvl + kvh) * (int64_t)d;
+            double *dvj = dv + (t * Hkvl + kvh) * (int64_t)d;
+            for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+            for (int g = 0; g < G; ++g) {
+                const int h = kvh * G + g;
+                for (int64_t i = j; i < de[j]; ++i) {
+                    const uint16_t *qi = q + (i * Hl + h) * (int64_t)d;
+                    const uint16_t *gi = dout + (i * Hl + h) * (int64_t)d;
+                    double s = 0.0, dp = 0.0;
+                    for (int c = 0; c < d; ++c) {
+                        s += bf16_to_f64(qi[c]) * bf16_to_f64(kj[c]);
+                        dp += bf16_to_f64(gi[c]) * bf16_to_f64(vj[c]);
+                    }
+                    const double p = exp(scale * s - LSE[(int64_t)h * N + i]);
+                    const double dsij = p * (dp - D[(int64_t)h * N + i]);
+                    for (int c = 0; c < d; ++c) {
+                        dvj[c] += p * bf16_to_f64(gi[c]);
+                        dkj[c] += scale * dsij * bf16_to_f64(qi[c]);
+                    }
+                }
+            }
+        }
+
+done:
+    free(ds); free(de); free(need); free(LSE); free(D);
+    return err;
+}

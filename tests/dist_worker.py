@@ -35,7 +35,8 @@ def _run(rank, world, case, out_q):
         from long_context_sequence_ulysses_b200 import dist as udist
         from workloads import random_case
 
-        c = random_case(case["N"], case["H"], case["Hkv"], case["d"], case["lengths"], seed=case["seed"])
+        c = random_case(case["N"], case["H"], case["Hkv"], case["d"], case["lengths"], seed=case["seed"],
+                        with_grad_out=bool(case.get("backward")))
         N, d = case["N"], case["d"]
         n_loc = N // world
         sl = slice(rank * n_loc, (rank + 1) * n_loc)
@@ -54,6 +55,20 @@ def _run(rank, world, case, out_q):
 
         args = (c["q"][sl].contiguous(), c["k"][sl].contiguous(), c["v"][sl].contiguous(),
                 c["position_ids"][sl].contiguous())
+        if case.get("backward"):
+            def attn_bwd(q, k, v, o, g, lse, pos, scale=None):
+                # the oracle recomputes O and LSE itself from q, k, v
+                dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, g, pos, scale=scale)
+                return tuple(torch.from_numpy(x).to(torch.bfloat16) for x in (dq, dk, dv))
+
+            o_loc, lse, pos, saved = udist.attention_forward(*args, attn=attn, pack=pack, unpack=unpack,
+                                                             keep_for_backward=True)
+            dq, dk, dv = udist.attention_backward(saved, lse, pos, c["do"][sl].contiguous(), attn_bwd=attn_bwd,
+                                                  pack=pack, unpack=unpack)
+            out_q.put((rank, o_loc.view(torch.int16).numpy().copy(),
+                       [x.view(torch.int16).numpy().copy() for x in (dq, dk, dv)], pos.numpy().copy(), None))
+            dist.barrier()
+            return
         if case.get("chunks"):
             o_loc, lse, pos, heads = udist.attention_forward_chunked(*args, case["chunks"], attn=attn, pack=pack,
                                                                      unpack=unpack)

@@ -75,3 +75,25 @@ def test_head_chunked_exchange_matches_unsharded(world, chunks):
     case = {"N": 64, "H": 16, "Hkv": 8, "d": 32, "lengths": [30, 2, 32], "seed": 5, "chunks": chunks}
     results = _run_world(world, case)
     _check_against_unsharded(world, case, results)
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_backward_exchange_matches_unsharded(world):
+    """The backward across ranks: dO crosses the first exchange, each rank
+    computes the gradients of its heads, dQ/dK/dV cross the second exchange
+    back to sequence shards. Every rank's shards of dQ, dK and dV equal the
+    unsharded oracle's gradients (rounded to bf16) bit for bit."""
+    case = {"N": 64, "H": 8, "Hkv": 4, "d": 16, "lengths": [23, 1, 40], "seed": 19, "backward": True}
+    results = _run_world(world, case)
+    c = random_case(case["N"], case["H"], case["Hkv"], case["d"], case["lengths"], seed=case["seed"],
+                    with_grad_out=True)
+    rq, rk, rv, ro, _ = oracle.attn_bwd(c["q"], c["k"], c["v"], c["do"], c["position_ids"])
+    bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy()
+    n_loc = case["N"] // world
+    for r in range(world):
+        o, (dq, dk, dv), pos, _ = results[r]
+        sl = slice(r * n_loc, (r + 1) * n_loc)
+        assert np.array_equal(o, bits(ro)[sl])
+        assert np.array_equal(dq, bits(rq)[sl])
+        assert np.array_equal(dk, bits(rk)[sl])
+        assert np.array_equal(dv, bits(rv)[sl])

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_grad_close, bf16_to_f64
+from helpers import assert_close, assert_grad_close, bf16_to_f64
 from workloads import WORKLOADS, make_inputs, random_case
 
 pytestmark = pytest.mark.gpu
@@ -81,9 +81,7 @@ def test_bwd_empty():
     assert dq.shape == (0, 2, 128)
 
 
-def test_train_workload_documents():
-    """Rank 0 of the training workload, through the same launches the
-    benchmark times; whole documents compared against the oracle."""
+def _train_rank0():
     import long_context_sequence_ulysses_b200 as U
     w = WORKLOADS["train"]
     inp = make_inputs(w, device="cuda", with_grad_out=True)
@@ -95,14 +93,26 @@ def test_train_workload_documents():
     o, lse = U.attn_fwd(q, k, v, pos)
     dq, dk, dv = U.attn_bwd(q, k, v, o, do, lse, pos)
     torch.cuda.synchronize()
-    lengths = np.array(inp["lengths"])
+    return w, inp, (q, k, v, do, pos), (dq, dk, dv)
+
+
+def _doc_bounds(lengths):
+    lengths = np.array(lengths)
     starts = np.concatenate([[0], np.cumsum(lengths)[:-1]])
-    # first, last, shortest and a mid-length document (skipping very long ones)
-    cand = [0, len(lengths) - 1, int(np.argmin(lengths))]
+    return lengths, starts
+
+
+def test_train_workload_documents():
+    """Rank 0 of the training workload, through the same launches the
+    benchmark times; whole documents compared against the oracle."""
+    w, inp, (q, k, v, do, pos), (dq, dk, dv) = _train_rank0()
+    lengths, starts = _doc_bounds(inp["lengths"])
+    # first, last-but-longest, shortest and a mid-length document, in full
+    cand = [0, int(np.argmin(lengths))]
     order = np.argsort(lengths)
     cand.append(int(order[len(order) // 2]))
     picked = sorted({t for t in cand if lengths[t] <= 9000})
-    assert picked
+    assert len(picked) >= 3
     for t in picked:
         a, b = int(starts[t]), int(starts[t] + lengths[t])
         sl = slice(a, b)
@@ -110,6 +120,99 @@ def test_train_workload_documents():
         assert_grad_close(f"dQ doc {t}", bf16_to_f64(dq[sl]), rq)
         assert_grad_close(f"dK doc {t}", bf16_to_f64(dk[sl]), rk)
         assert_grad_close(f"dV doc {t}", bf16_to_f64(dv[sl]), rv)
+
+
+def test_train_longest_document():
+    """The longest document of the training workload (18112 tokens): the dK/dV
+    of its first 256 keys (the key tiles that every later query of the document
+    reaches, the longest-running dK/dV work), of its last keys and of random
+    keys, and the dQ of its last 128-row tile and random rows, against the
+    oracle's exact gradients at those keys and rows."""
+    w, inp, (q, k, v, do, pos), (dq, dk, dv) = _train_rank0()
+    lengths, starts = _doc_bounds(inp["lengths"])
+    t = int(np.argmax(lengths))
+    a, L = int(starts[t]), int(lengths[t])
+    assert L > 9000
+    rng = np.random.default_rng(3)
+    keys = np.unique(np.concatenate([np.arange(256), np.arange(L - 16, L), rng.integers(0, L, 48)]))
+    rows = np.unique(np.concatenate([np.arange(8), np.arange(L - 128, L), rng.integers(0, L, 48)]))
+    sl = slice(a, a + L)
+    rq, rk, rv = oracle.attn_bwd_sampled(q[sl].cpu(), k[sl].cpu(), v[sl].cpu(), do[sl].cpu(), pos[sl].cpu(),
+                                         rows, keys)
+    kt, rt = torch.from_numpy(keys + a).cuda(), torch.from_numpy(rows + a).cuda()
+    assert_grad_close("dK longest doc", bf16_to_f64(dk[kt]), rk)
+    assert_grad_close("dV longest doc", bf16_to_f64(dv[kt]), rv)
+    assert_grad_close("dQ longest doc", bf16_to_f64(dq[rt]), rq)
+
+
+def test_train_fused_all_ranks():
+    """The fused forward and backward as the benchmark's fused step runs them
+    on the training workload: every one of the 4 ranks reads its 8 query heads
+    and 2 KV heads straight out of the sequence-sharded buffers and writes O and
+    dQ/dK/dV into the sequence layout. One document per rank (one straddling a
+    128-token tile boundary, one long one on rank 1) against the oracle on that
+    rank's head slice of the inputs."""
+    import long_context_sequence_ulysses_b200 as U
+    w = WORKLOADS["train"]
+    inp = make_inputs(w, device="cuda", with_grad_out=True)
+    pos = inp["position_ids"]
+    nan = float("nan")
+    o_seq = torch.full_like(inp["q"], nan)
+    dq_s, dk_s, dv_s = (torch.full_like(inp[x], nan) for x in ("q", "k", "v"))
+    lse_all = torch.empty((w.H, w.N), dtype=torch.float32, device="cuda")
+    for r in range(w.P):
+        U.attn_fwd_fused(inp["q"], inp["k"], inp["v"], pos, w.P, r, out=o_seq, lse=lse_all[r * w.Hl:(r + 1) * w.Hl])
+    for r in range(w.P):
+        U.attn_bwd_fused(inp["q"], inp["k"], inp["v"], o_seq, inp["do"], lse_all[r * w.Hl:(r + 1) * w.Hl], pos,
+                         w.P, r, dq=dq_s, dk=dk_s, dv=dv_s)
+    torch.cuda.synchronize()
+    for x in (o_seq, dq_s, dk_s, dv_s):
+        assert not torch.isnan(x.float()).any()          # the ranks together wrote every head
+    lengths, starts = _doc_bounds(inp["lengths"])
+    cpu = {x: inp[x].cpu() for x in ("q", "k", "v", "do")}
+    pc = pos.cpu()
+    full_docs = {0: 3, 2: 7, 3: 1}       # 240 tokens across a tile boundary, 1127, 1280
+    for r in range(w.P):
+        qs, ks = slice(r * w.Hl, (r + 1) * w.Hl), slice(r * w.Hkvl, (r + 1) * w.Hkvl)
+        if r in full_docs:
+            t = full_docs[r]
+            a, b = int(starts[t]), int(starts[t] + lengths[t])
+            sl = slice(a, b)
+            rq, rk, rv, ro, rl = oracle.attn_bwd(cpu["q"][sl, qs].contiguous(), cpu["k"][sl, ks].contiguous(),
+                                                 cpu["v"][sl, ks].contiguous(), cpu["do"][sl, qs].contiguous(), pc[sl])
+            assert_close(f"O rank {r}", bf16_to_f64(o_seq[sl, qs]), ro)
+            assert_close(f"LSE rank {r}", lse_all[qs, a:b].double().cpu().numpy(), rl)
+            assert_grad_close(f"dQ fused rank {r}", bf16_to_f64(dq_s[sl, qs]), rq)
+            assert_grad_close(f"dK fused rank {r}", bf16_to_f64(dk_s[sl, ks]), rk)
+            assert_grad_close(f"dV fused rank {r}", bf16_to_f64(dv_s[sl, ks]), rv)
+        else:
+            t = 8                        # 9120 tokens: sampled keys and rows
+            a, L = int(starts[t]), int(lengths[t])
+            rng = np.random.default_rng(r)
+            keys = np.unique(np.concatenate([np.arange(128), rng.integers(0, L, 32)]))
+            rows = np.unique(np.concatenate([np.arange(L - 128, L), rng.integers(0, L, 32)]))
+            sl = slice(a, a + L)
+            rq, rk, rv = oracle.attn_bwd_sampled(cpu["q"][sl, qs].contiguous(), cpu["k"][sl, ks].contiguous(),
+                                                 cpu["v"][sl, ks].contiguous(), cpu["do"][sl, qs].contiguous(),
+                                                 pc[sl], rows, keys)
+            kt, rt = torch.from_numpy(keys + a).cuda(), torch.from_numpy(rows + a).cuda()
+            assert_grad_close(f"dK fused rank {r}", bf16_to_f64(dk_s[kt][:, ks]), rk)
+            assert_grad_close(f"dV fused rank {r}", bf16_to_f64(dv_s[kt][:, ks]), rv)
+            assert_grad_close(f"dQ fused rank {r}", bf16_to_f64(dq_s[rt][:, qs]), rq)
+
+
+@pytest.mark.parametrize("kind", ["first_not_zero", "jumps_repeats_negatives"])
+def test_bwd_irregular_position_ids(kind):
+    from test_gpu_attn_fwd import _irregular_ids
+    N, Hl, Hkvl, d = 1000, 4, 2, 128
+    c = random_case(N, Hl, Hkvl, d, [N], seed=71, device="cuda", with_grad_out=True)
+    pos = _irregular_ids(kind, N)
+    c["position_ids"] = pos.cuda()
+    _, _, dq, dk, dv = _fwd_bwd(c)
+    rq, rk, rv, _, _ = oracle.attn_bwd(c["q"], c["k"], c["v"], c["do"], pos)
+    assert_grad_close("dQ", bf16_to_f64(dq), rq)
+    assert_grad_close("dK", bf16_to_f64(dk), rk)
+    assert_grad_close("dV", bf16_to_f64(dv), rv)
 
 
 def test_bwd_fused_equals_slice():

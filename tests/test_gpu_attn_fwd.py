@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_close, bf16_to_f64, sample_rows
+from helpers import assert_close, bf16_to_f64, sample_rows, stratified_long_rows
 from workloads import WORKLOADS, make_inputs, random_case
 
 pytestmark = pytest.mark.gpu
@@ -132,13 +132,17 @@ def test_fwd_empty():
     assert o.shape == (0, 2, 128) and lse.shape == (2, 0)
 
 
-WORKLOAD_SAMPLES = {"tiny": None, "llama8b": 160, "long131k": 24, "million": 6, "train": 160}
+WORKLOAD_SAMPLES = {"tiny": None, "llama8b": 160, "train": 160}
+# Single long documents: (tile stride of the first/last-row strata, extra uniform rows).
+# long131k: both edge rows of all 1024 tiles; million: of every 32nd of its 8192 tiles.
+LONG_STRATA = {"long131k": (1, 64), "million": (32, 32)}
 
 
 @pytest.mark.parametrize("name", ["tiny", "llama8b", "long131k", "million", "train"])
 def test_workload_forward(name):
     """Rank 0's head slice of each workload, produced by the seq->head exchange
-    and run through the same forward launch the benchmark times."""
+    and run through the same forward launch the benchmark times. Every sampled
+    row is compared on all of rank 0's heads, exact over all its keys."""
     import long_context_sequence_ulysses_b200 as U
     w = WORKLOADS[name]
     inp = make_inputs(w, device="cuda", with_grad_out=False)
@@ -149,16 +153,72 @@ def test_workload_forward(name):
     del inp["q"], inp["k"], inp["v"]
     o, lse = U.attn_fwd(q, k, v, inp["position_ids"])
     torch.cuda.synchronize()
-    n_rand = WORKLOAD_SAMPLES[name]
-    if n_rand is None:
+    if name in LONG_STRATA:
+        stride, n_rand = LONG_STRATA[name]
+        rows = stratified_long_rows(w.N, stride, n_rand, seed=w.seed)
+        assert len(rows) >= 256
+    elif WORKLOAD_SAMPLES[name] is None:
         rows = np.arange(w.N)
     else:
-        rows = sample_rows(inp["lengths"], w.N, n_rand, seed=w.seed)
-        if name in ("long131k", "million"):
-            # single long document: keep the sample affordable but include the far end
-            rng = np.random.default_rng(w.seed)
-            rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1], rng.integers(0, w.N, n_rand)]))
+        rows = sample_rows(inp["lengths"], w.N, WORKLOAD_SAMPLES[name], seed=w.seed)
     rt = torch.from_numpy(rows).cuda()
     ro, rl = oracle.attn_fwd(q.cpu(), k.cpu(), v.cpu(), inp["position_ids"].cpu(), rows=rows)
+    assert ro.shape[1] == w.Hl
     assert_close("O", bf16_to_f64(o[rt]), ro)
     assert_close("LSE", lse[:, rt].double().cpu().numpy(), rl)
+
+
+def test_fused_forward_llama8b_all_ranks():
+    """The fused forward as the benchmark's fused step runs it on llama8b: every
+    one of the 8 ranks reads its 4 query heads and 1 KV head straight out of the
+    sequence-sharded Q/K/V (rows 8 KB and 2 KB apart) and writes its heads of
+    O into the sequence layout. Sampled rows of every rank, all of its heads,
+    against the oracle on that rank's head slice of the inputs."""
+    import long_context_sequence_ulysses_b200 as U
+    w = WORKLOADS["llama8b"]
+    inp = make_inputs(w, device="cuda", with_grad_out=False)
+    pos = inp["position_ids"]
+    o_seq = torch.full_like(inp["q"], float("nan"))
+    lse_all = torch.empty((w.H, w.N), dtype=torch.float32, device="cuda")
+    for r in range(w.P):
+        U.attn_fwd_fused(inp["q"], inp["k"], inp["v"], pos, w.P, r, out=o_seq,
+                         lse=lse_all[r * w.Hl:(r + 1) * w.Hl])
+    torch.cuda.synchronize()
+    assert not torch.isnan(o_seq.float()).any()          # every rank wrote exactly its own heads
+    qc, kc, vc, pc = inp["q"].cpu(), inp["k"].cpu(), inp["v"].cpu(), pos.cpu()
+    for r in range(w.P):
+        rows = sample_rows(inp["lengths"], w.N, 48, seed=100 + r)
+        qs, ks = slice(r * w.Hl, (r + 1) * w.Hl), slice(r * w.Hkvl, (r + 1) * w.Hkvl)
+        ro, rl = oracle.attn_fwd(qc[:, qs].contiguous(), kc[:, ks].contiguous(), vc[:, ks].contiguous(), pc,
+                                 rows=rows)
+        rt = torch.from_numpy(rows).cuda()
+        assert_close(f"O rank {r}", bf16_to_f64(o_seq[rt][:, qs]), ro)
+        assert_close(f"LSE rank {r}", lse_all[qs][:, rt].double().cpu().numpy(), rl)
+
+
+def _irregular_ids(kind: str, N: int) -> torch.Tensor:
+    """Position ids that break the 0, 1, 2, ... pattern in the ways the reading
+    of the ids has to handle (a document starts at token 0 and at every 0;
+    every other value is ignored)."""
+    if kind == "first_not_zero":       # a shard boundary inside a document: ids start at 300
+        ids = list(range(300, 300 + 700)) + list(range(N - 700))
+    elif kind == "no_zero_at_all":     # one document, ids never 0
+        ids = [7 + i for i in range(N)]
+    else:                              # jumps, repeats and negative ids between the zeros
+        ids = (list(range(100)) + list(range(500, 640)) + [3] * 40 + list(range(160)) + [-1] * 30
+               + list(range(129)) + [9] * 3 + list(range(N - 602)))
+    assert len(ids) == N
+    return torch.tensor(ids, dtype=torch.int32)
+
+
+@pytest.mark.parametrize("kind", ["first_not_zero", "no_zero_at_all", "jumps_repeats_negatives"])
+@pytest.mark.parametrize("Hl,Hkvl,d", [(4, 2, 128), (3, 1, 64)])
+def test_fwd_irregular_position_ids(kind, Hl, Hkvl, d):
+    N = 1000
+    c = random_case(N, Hl, Hkvl, d, [N], seed=61 + Hl, device="cuda")
+    pos = _irregular_ids(kind, N)
+    c["position_ids"] = pos.cuda()
+    o, lse = _run(c)
+    ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], pos)
+    assert_close("O", bf16_to_f64(o), ro)
+    assert_close("LSE", lse.double().cpu().numpy(), rl)

@@ -337,3 +337,56 @@ def test_bwd_sum_rules_per_document():
                                        g[a:b, kvh * G:(kvh + 1) * G].sum(axis=(0, 1)), atol=1e-11)
     o2, l2 = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
     assert np.array_equal(o, o2) and np.array_equal(lse, l2)
+
+
+# Position ids that do not count 0, 1, 2, ... from token 0: the first document
+# starts at token 0 whatever its id, every later 0 starts a new document, and
+# any other value (a jump, a repeat, a negative id) is ignored.
+IRREGULAR_POS = [5, 6, 7, 0, 1, 9, 9, -3, 0, 2, 0, 1, 1, 4]
+
+
+def test_bwd_sampled_matches_full():
+    """The sampled backward equals the full backward on the rows and keys it is
+    asked for (first and last keys of documents, a one-token document, GQA)."""
+    lengths = [40, 1, 55, 32]
+    N, H, Hkv, d = sum(lengths), 6, 2, 16
+    c = random_case(N, H, Hkv, d, lengths, seed=17, with_grad_out=True)
+    dq, dk, dv, _, _ = oracle.attn_bwd(c["q"], c["k"], c["v"], c["do"], c["position_ids"])
+    rows = [0, 3, 39, 40, 41, 95, 96, 127]
+    keys = [0, 1, 39, 40, 41, 42, 94, 95, 96, 120, 127]
+    sq, sk, sv = oracle.attn_bwd_sampled(c["q"], c["k"], c["v"], c["do"], c["position_ids"], rows, keys)
+    assert np.array_equal(sq, dq[rows])
+    assert np.array_equal(sk, dk[keys]) and np.array_equal(sv, dv[keys])
+
+
+def test_bwd_sampled_matches_autograd_irregular_ids():
+    """Against torch autograd of the explicit masked attention, with position
+    ids that start above 0, jump, repeat and go negative."""
+    pos = np.array(IRREGULAR_POS, dtype=np.int32)
+    N, H, Hkv, d = len(pos), 4, 2, 8
+    c = random_case(N, H, Hkv, d, [N], seed=23, with_grad_out=True)
+    c["position_ids"] = torch.from_numpy(pos)
+    scale = 1.0 / math.sqrt(d)
+    q = c["q"].double().requires_grad_()
+    k = c["k"].double().requires_grad_()
+    v = c["v"].double().requires_grad_()
+    out = _torch_attention_f64(q, k, v, pos, scale)
+    (out * c["do"].double()).sum().backward()
+    rows = list(range(N))
+    sq, sk, sv = oracle.attn_bwd_sampled(c["q"], c["k"], c["v"], c["do"], c["position_ids"], rows, rows)
+    np.testing.assert_allclose(sq, q.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(sk, k.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(sv, v.grad.numpy(), atol=1e-11, rtol=0)
+    dq, dk, dv, o, _ = oracle.attn_bwd(c["q"], c["k"], c["v"], c["do"], c["position_ids"])
+    np.testing.assert_allclose(o, out.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dk, k.grad.numpy(), atol=1e-11, rtol=0)
+
+
+def test_fwd_irregular_ids_match_brute_force():
+    pos = np.array(IRREGULAR_POS, dtype=np.int32)
+    N, H, Hkv, d = len(pos), 4, 1, 8
+    c = random_case(N, H, Hkv, d, [N], seed=29)
+    o, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], pos)
+    bo, bl = brute_attention(f64(c["q"]), f64(c["k"]), f64(c["v"]), pos, 1.0 / math.sqrt(d))
+    np.testing.assert_allclose(o, bo, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, bl, atol=1e-12, rtol=0)

@@ -2,9 +2,10 @@
 device memory (for example a plugin whose host framework owns every device
 buffer and hands over only inputs and outputs). Its scratch lives in a static
 device array inside the library. Called here through the C ABI and compared
-with ulysses_attn_fwd (which takes a caller-provided workspace) on two calls
-in a row, so stale scratch left by the first call would show up in the
-second. Collected last on purpose."""
+with ulysses_attn_fwd (which takes a caller-provided workspace) on three calls
+in a row (two whose schedule pairs heads, then one whose schedule pairs query
+tiles), so stale scratch left by one call would show up in the next.
+Collected last on purpose."""
 import ctypes
 
 import pytest
@@ -30,12 +31,15 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def test_noalloc_matches_attn_fwd_on_two_calls():
+def test_noalloc_matches_attn_fwd_on_consecutive_calls():
     U, lib, f = _fn()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     cases = [
         random_case(3000, 4, 2, 128, [1200, 1, 1799], seed=41, device="cuda"),
         random_case(1536, 2, 1, 64, [700, 300, 536], seed=42, device="cuda"),
+        # odd group size: the schedule holds pairs of query tiles (a different
+        # layout of the same scratch), N not a multiple of 256
+        random_case(2000, 3, 1, 128, [1500, 2, 498], seed=43, device="cuda"),
     ]
     for c in cases:
         N, Hl, d = c["q"].shape
