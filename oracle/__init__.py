@@ -13,6 +13,8 @@ Parity status of each function (what pins it is listed in the tests):
   attn_fwd                  pinned (brute force, SDPA, closed forms, invariances)
   attn_bwd                  pinned (finite differences, autograd, sum rules)
   attn_bwd_sampled          pinned (equal to attn_bwd on the sampled rows and keys)
+  attn_fwd_window           pinned (brute force with the window, whole window = attn_fwd)
+  merge                     pinned (closed form; merged windows = attention over their union)
 """
 from __future__ import annotations
 
@@ -61,6 +63,10 @@ def _load():
             lib.oracle_attn_bwd.restype = I32
             lib.oracle_attn_bwd_sampled.argtypes = [P, P, P, P, P, I64, I32, I32, I32, F64, P, I64, P, I64, P, P, P]
             lib.oracle_attn_bwd_sampled.restype = I32
+            lib.oracle_attn_fwd_window_rows.argtypes = [P, P, P, P, I64, I32, I32, I32, F64, I64, I64, P, I64, P, P]
+            lib.oracle_attn_fwd_window_rows.restype = I32
+            lib.oracle_merge.argtypes = [P, P, I32, I64, I32, I32, P, P]
+            lib.oracle_merge.restype = None
             _lib = lib
     return _lib
 
@@ -187,3 +193,38 @@ def attn_bwd_sampled(q, k, v, dout, pos, rows: Sequence[int], keys: Sequence[int
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd_sampled failed ({rc})")
     return dq, dk, dv
+
+
+def attn_fwd_window(q, k, v, pos, kv_lo: int, kv_hi: int, scale: Optional[float] = None,
+                    rows: Optional[Sequence[int]] = None):
+    """Attention of one rank's head slice over the keys [kv_lo, kv_hi) only
+    (one ring step's partial result). Returns (o [rows][Hl][d], lse [Hl][rows])
+    in fp64; a row that sees no key gets o = 0, lse = -inf."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    N, Hl, d = qb.shape
+    Hkvl = kb.shape[1]
+    p = _i32(pos)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    nr = r.shape[0]
+    o = np.empty((Hl, nr, d), dtype=np.float64)
+    lse = np.empty((Hl, nr), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_window_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(p), N, Hl, Hkvl, d, float(scale),
+                                             int(kv_lo), int(kv_hi), _ptr(r), nr, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd_window_rows failed ({rc})")
+    return np.ascontiguousarray(o.transpose(1, 0, 2)), lse
+
+
+def merge(o_parts, lse_parts):
+    """Merge partial results over disjoint key sets: o_parts [R][M][Hl][d],
+    lse_parts [R][Hl][M] (fp64) -> (o [M][Hl][d], lse [Hl][M])."""
+    op = np.ascontiguousarray(o_parts, dtype=np.float64)
+    lp = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    R, M, Hl, d = op.shape
+    assert lp.shape == (R, Hl, M)
+    o = np.empty((M, Hl, d), dtype=np.float64)
+    lse = np.empty((Hl, M), dtype=np.float64)
+    _load().oracle_merge(_ptr(op), _ptr(lp), R, M, Hl, d, _ptr(o), _ptr(lse))
+    return o, lse

@@ -418,3 +418,111 @@ done:
     free(ds); free(de); free(need); free(LSE); free(D);
     return err;
 }
+
+/* ------------------------------------------------------------------------ */
+/* ring steps: attention over a key window, and the merge of partial results */
+/* ------------------------------------------------------------------------ */
+
+/* Ring attention (set against Ulysses on the page "Ulysses 序列並行：百萬 Token
+ * 上下文訓練", section "競品分析", and on the page "Ulysses verteilt
+ * Millionen-Token-Kontexte auf mehrere GPUs", section "Wann Ulysses sinnvoll
+ * ist") passes the keys and values around the ranks chunk by chunk; each step
+ * gives the attention of the local queries over one chunk of keys. That
+ * partial result is the ordinary attention restricted to the keys of the
+ * window [kv_lo, kv_hi): row i sees keys j in [max(doc_start(i), kv_lo),
+ * min(i, kv_hi - 1)]. A row that sees no key gets o = 0 and lse = -inf.
+ * rows[nrows] are query indices; o is [Hl][nrows][d], lse is [Hl][nrows].   */
+int oracle_attn_fwd_window_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                const int32_t *pos, int64_t N, int Hl, int Hkvl, int d,
+                                double scale, int64_t kv_lo, int64_t kv_hi,
+                                const int64_t *rows, int64_t nrows, double *o, double *lse)
+{
+    if (Hkvl <= 0 || Hl % Hkvl != 0) return -1;
+    int32_t *ds = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
+    if (!ds) return -2;
+    oracle_doc_start(pos, N, ds);
+    const int G = Hl / Hkvl;
+    int err = 0;
+    #pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        if (!s_buf) {
+            #pragma omp atomic write
+            err = -2;
+        } else {
+            #pragma omp for collapse(2) schedule(dynamic, 4)
+            for (int h = 0; h < Hl; ++h)
+                for (int64_t r = 0; r < nrows; ++r) {
+                    const int64_t i = rows[r];
+                    const int64_t lo = ds[i] > kv_lo ? ds[i] : kv_lo;
+                    const int64_t hi = i < kv_hi - 1 ? i : kv_hi - 1;
+                    double *orow = o + (h * nrows + r) * (int64_t)d;
+                    double *l_out = lse + h * nrows + r;
+                    if (lo > hi) {
+                        for (int c = 0; c < d; ++c) orow[c] = 0.0;
+                        *l_out = -INFINITY;
+                        continue;
+                    }
+                    const int kvh = h / G;
+                    const uint16_t *qi = q + (i * Hl + h) * (int64_t)d;
+                    double m = -INFINITY;
+                    for (int64_t j = lo; j <= hi; ++j) {
+                        const uint16_t *kj = k + (j * Hkvl + kvh) * (int64_t)d;
+                        double acc = 0.0;
+                        for (int c = 0; c < d; ++c) acc += bf16_to_f64(qi[c]) * bf16_to_f64(kj[c]);
+                        acc *= scale;
+                        s_buf[j - lo] = acc;
+                        if (acc > m) m = acc;
+                    }
+                    double l = 0.0;
+                    for (int c = 0; c < d; ++c) orow[c] = 0.0;
+                    for (int64_t j = lo; j <= hi; ++j) {
+                        const double e = exp(s_buf[j - lo] - m);
+                        l += e;
+                        const uint16_t *vj = v + (j * Hkvl + kvh) * (int64_t)d;
+                        for (int c = 0; c < d; ++c) orow[c] += e * bf16_to_f64(vj[c]);
+                    }
+                    for (int c = 0; c < d; ++c) orow[c] /= l;
+                    *l_out = m + log(l);
+                }
+            free(s_buf);
+        }
+    }
+    free(ds);
+    return err;
+}
+
+/* The merge of R partial results over disjoint key sets into the result over
+ * their union: with L = log sum_s exp(lse_s), o = sum_s exp(lse_s - L) o_s and
+ * lse = L (each partial o_s is already normalised by its own sum exp(lse_s)).
+ * A partial with lse_s = -inf (no key) contributes nothing; if every one is
+ * -inf, o = 0 and lse = -inf.
+ * o_parts [R][M][Hl][d], lse_parts [R][Hl][M]; o [M][Hl][d], lse [Hl][M].  */
+void oracle_merge(const double *o_parts, const double *lse_parts, int R, int64_t M, int Hl, int d,
+                  double *o, double *lse)
+{
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int h = 0; h < Hl; ++h)
+        for (int64_t m = 0; m < M; ++m) {
+            double mx = -INFINITY;
+            for (int s = 0; s < R; ++s) {
+                const double x = lse_parts[((int64_t)s * Hl + h) * M + m];
+                if (x > mx) mx = x;
+            }
+            double *orow = o + (m * Hl + h) * (int64_t)d;
+            for (int c = 0; c < d; ++c) orow[c] = 0.0;
+            if (mx == -INFINITY) {
+                lse[(int64_t)h * M + m] = -INFINITY;
+                continue;
+            }
+            double sum = 0.0;
+            for (int s = 0; s < R; ++s) sum += exp(lse_parts[((int64_t)s * Hl + h) * M + m] - mx);
+            const double L = mx + log(sum);
+            for (int s = 0; s < R; ++s) {
+                const double w = exp(lse_parts[((int64_t)s * Hl + h) * M + m] - L);
+                const double *op = o_parts + (((int64_t)s * M + m) * Hl + h) * (int64_t)d;
+                for (int c = 0; c < d; ++c) orow[c] += w * op[c];
+            }
+            lse[(int64_t)h * M + m] = L;
+        }
+}

@@ -390,3 +390,85 @@ def test_fwd_irregular_ids_match_brute_force():
     bo, bl = brute_attention(f64(c["q"]), f64(c["k"]), f64(c["v"]), pos, 1.0 / math.sqrt(d))
     np.testing.assert_allclose(o, bo, atol=1e-12, rtol=0)
     np.testing.assert_allclose(lse, bl, atol=1e-12, rtol=0)
+
+
+# --------------------------------------------------------------------- ring steps
+
+def _brute_window(q, k, v, pos, scale, kv_lo, kv_hi):
+    """brute_attention with the keys further restricted to [kv_lo, kv_hi);
+    rows that see no key get o = 0, lse = -inf."""
+    N, Hl, d = q.shape
+    G = Hl // k.shape[1]
+    mask = same_doc_mask(np.asarray(pos))
+    cols = np.arange(N)
+    mask &= ((cols >= kv_lo) & (cols < kv_hi))[None, :]
+    o = np.zeros((N, Hl, d))
+    lse = np.full((Hl, N), -np.inf)
+    for h in range(Hl):
+        s = scale * (q[:, h, :] @ k[:, h // G, :].T)
+        for i in range(N):
+            if not mask[i].any():
+                continue
+            si = s[i][mask[i]]
+            mx = si.max()
+            e = np.exp(si - mx)
+            o[i, h] = (e / e.sum()) @ v[mask[i], h // G, :]
+            lse[h, i] = mx + np.log(e.sum())
+    return o, lse
+
+
+@pytest.mark.parametrize("kv_lo,kv_hi", [(0, 45), (8, 16), (13, 30), (20, 20), (44, 45), (0, 1)])
+def test_window_matches_brute_force(kv_lo, kv_hi):
+    lengths = [12, 1, 20, 12]
+    N, H, Hkv, d = sum(lengths), 4, 2, 8
+    c = random_case(N, H, Hkv, d, lengths, seed=37)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = oracle.attn_fwd_window(c["q"], c["k"], c["v"], c["position_ids"], kv_lo, kv_hi)
+    bo, bl = _brute_window(f64(c["q"]), f64(c["k"]), f64(c["v"]), c["position_ids"].numpy(), scale, kv_lo, kv_hi)
+    np.testing.assert_allclose(o, bo, atol=1e-12, rtol=0)
+    assert np.array_equal(np.isinf(lse), np.isinf(bl))
+    np.testing.assert_allclose(lse[np.isfinite(lse)], bl[np.isfinite(bl)], atol=1e-12, rtol=0)
+
+
+def test_window_over_all_keys_equals_attention():
+    lengths = [30, 2, 33]
+    N = sum(lengths)
+    c = random_case(N, 4, 1, 16, lengths, seed=41)
+    o, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    ow, lw = oracle.attn_fwd_window(c["q"], c["k"], c["v"], c["position_ids"], 0, N)
+    assert np.array_equal(o, ow) and np.array_equal(lse, lw)
+
+
+def test_merge_closed_form():
+    """Two partials with sums e^a and e^b: the merged output is their average
+    weighted by those sums, and the merged lse is log(e^a + e^b); a partial
+    with lse = -inf contributes nothing; all -inf gives o = 0, lse = -inf."""
+    a, b = 0.3, -1.7
+    x = np.array([1.0, -2.0, 0.5])
+    y = np.array([4.0, 0.25, -1.0])
+    o_parts = np.zeros((3, 3, 1, 3))
+    lse_parts = np.full((3, 1, 3), -np.inf)
+    o_parts[0, 0, 0], o_parts[1, 0, 0], lse_parts[0, 0, 0], lse_parts[1, 0, 0] = x, y, a, b
+    o_parts[1, 1, 0], lse_parts[1, 0, 1] = y, b          # row 1: only the second partial sees keys
+    o, lse = oracle.merge(o_parts, lse_parts)
+    ea, eb = math.exp(a), math.exp(b)
+    np.testing.assert_allclose(o[0, 0], (ea * x + eb * y) / (ea + eb), atol=1e-15)
+    assert lse[0, 0] == pytest.approx(math.log(ea + eb), abs=1e-15)
+    np.testing.assert_allclose(o[1, 0], y, atol=1e-15)
+    assert lse[0, 1] == pytest.approx(b, abs=1e-15)
+    assert np.all(o[2] == 0.0) and lse[0, 2] == -np.inf
+
+
+@pytest.mark.parametrize("bounds", [[0, 16, 32, 48, 65], [0, 5, 40, 65], [0, 65]])
+def test_merged_windows_equal_attention(bounds):
+    """Attention over disjoint key windows that cover every key, merged, is
+    the attention over all keys: the identity a ring of chunk steps relies on."""
+    lengths = [30, 2, 33]
+    N = sum(lengths)
+    c = random_case(N, 4, 2, 16, lengths, seed=43)
+    o, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    parts = [oracle.attn_fwd_window(c["q"], c["k"], c["v"], c["position_ids"], lo, hi)
+             for lo, hi in zip(bounds[:-1], bounds[1:])]
+    om, lm = oracle.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(om, o, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lm, lse, atol=1e-12, rtol=0)
