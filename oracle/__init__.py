@@ -228,3 +228,48 @@ def merge(o_parts, lse_parts):
     lse = np.empty((Hl, M), dtype=np.float64)
     _load().oracle_merge(_ptr(op), _ptr(lp), R, M, Hl, d, _ptr(o), _ptr(lse))
     return o, lse
+
+
+# ---------------------------------------------------------------- projections
+# The steps either side of the path (page "Hugging Face并行加速：10倍提升超长序列训练效率",
+# section "Ulysses的工作原理", steps QKV投影 and 输出投影; page "DeepSpeed Ulysses
+# 详解", section "DeepSpeed-Ulysses 的核心机制", items 2 and 6): every rank
+# projects its own tokens with the full weights. The product is numpy's fp64
+# matmul of the exactly widened bf16 values (a library primitive used as a
+# step); the exchange layout is the pinned seq_to_head / head_to_seq above.
+
+def _f64(x) -> np.ndarray:
+    b = _bits(x)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def qkv_proj(x, w_qkv, P: int, H: int, Hkv: int, d: int, rows: Optional[Sequence[int]] = None):
+    """x [N][hidden] (the P sequence shards), w_qkv [(H+2Hkv)*d][hidden] ->
+    fp64 (q, k, v) in every rank's head-slice layout [P][N][H/P][d] and
+    [P][N][Hkv/P][d]: y = x w_qkv^T, columns [0, H*d) are Q's heads, then K's,
+    then V's, each head's d columns contiguous. With ``rows``, only those
+    tokens: [P][len(rows)][heads/P][d]."""
+    xf = _f64(x)
+    if rows is not None:
+        xf = xf[np.asarray(rows, dtype=np.int64)]
+    y = xf @ _f64(w_qkv).T
+    n = y.shape[0]
+    out = []
+    for lo, heads in ((0, H), (H * d, Hkv), ((H + Hkv) * d, Hkv)):
+        part = y[:, lo:lo + heads * d].reshape(n, heads, d)
+        # the exchange: rank r holds heads [r*heads/P, (r+1)*heads/P) of every token
+        out.append(np.ascontiguousarray(part.reshape(n, P, heads // P, d).transpose(1, 0, 2, 3)))
+    return tuple(out)
+
+
+def out_proj(o_heads, w_o, rows: Optional[Sequence[int]] = None):
+    """o_heads [P][N][H/P][d] (every rank's head slice of the attention output),
+    w_o [hidden][H*d] -> y [N][hidden] fp64: the second exchange back to the
+    sequence layout [N][H*d] (head r*H/P + h at columns (r*H/P + h)*d ...), then
+    y = o w_o^T. With ``rows``, only those tokens."""
+    of = _f64(o_heads)
+    P, N, Hl, d = of.shape
+    seq = of.transpose(1, 0, 2, 3).reshape(N, P * Hl * d)
+    if rows is not None:
+        seq = seq[np.asarray(rows, dtype=np.int64)]
+    return seq @ _f64(w_o).T

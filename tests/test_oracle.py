@@ -472,3 +472,63 @@ def test_merged_windows_equal_attention(bounds):
     om, lm = oracle.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
     np.testing.assert_allclose(om, o, atol=1e-12, rtol=0)
     np.testing.assert_allclose(lm, lse, atol=1e-12, rtol=0)
+
+
+# --------------------------------------------------------------------- projections
+
+def _bf(shape, seed):
+    from workloads import normal_bf16
+    return normal_bf16(shape, seed)
+
+
+def test_qkv_proj_identity_weights_is_the_exchange():
+    """With w_qkv = [I; I; I] (hidden = H*d = Hkv*d), the projection returns x
+    itself as Q, K and V, and the layout is exactly seq_to_head's."""
+    N, P, H, d = 16, 2, 4, 8
+    x = _bf((N, H * d), 3)
+    eye = torch.eye(H * d, dtype=torch.bfloat16)
+    w = torch.cat([eye, eye, eye], 0)
+    q, k, v = oracle.qkv_proj(x, w, P, H, H, d)
+    ref = oracle.seq_to_head(x.view(N, H, d), N, P, H, d)
+    bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for t in (q, k, v):
+        assert np.array_equal(bits(t), ref)
+
+
+def test_qkv_proj_closed_form_and_head_order():
+    """One token, hand-built weights: column block j of w_qkv picks x[j] times
+    a known factor, so each head of Q, K, V holds a known value at a known
+    rank and position."""
+    P, H, Hkv, d = 2, 2, 2, 1          # hidden = 2, six output columns: q0 q1 k0 k1 v0 v1
+    x = torch.tensor([[1.5, -2.0]], dtype=torch.bfloat16)
+    w = torch.tensor([[1, 0], [0, 1], [2, 0], [0, 2], [1, 1], [1, -1]], dtype=torch.bfloat16)
+    q, k, v = oracle.qkv_proj(x, w, P, H, Hkv, d)
+    assert q.shape == (2, 1, 1, 1) and q[0, 0, 0, 0] == 1.5 and q[1, 0, 0, 0] == -2.0
+    assert k[0, 0, 0, 0] == 3.0 and k[1, 0, 0, 0] == -4.0
+    assert v[0, 0, 0, 0] == -0.5 and v[1, 0, 0, 0] == 3.5
+
+
+def test_out_proj_identity_weights_is_the_inverse_exchange():
+    P, N, Hl, d = 4, 8, 2, 4
+    o = _bf((P, N, Hl, d), 5)
+    y = oracle.out_proj(o, torch.eye(P * Hl * d, dtype=torch.bfloat16))
+    back = oracle.head_to_seq(o, N, P, P * Hl, d).reshape(N, P * Hl * d)
+    bits = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bits, back)
+
+
+def test_projections_against_torch_matmul():
+    N, P, H, Hkv, d, hidden = 12, 2, 4, 2, 8, 24
+    x, w = _bf((N, hidden), 7), _bf(((H + 2 * Hkv) * d, hidden), 8)
+    q, k, v = oracle.qkv_proj(x, w, P, H, Hkv, d)
+    y = x.double() @ w.double().T
+    np.testing.assert_allclose(q[1, :, 0], y[:, (H // P) * d:(H // P + 1) * d].numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(v[1, :, 0], y[:, (H + Hkv + Hkv // P) * d:(H + Hkv + Hkv // P + 1) * d].numpy(),
+                               rtol=0, atol=1e-12)
+    rows = [0, 5, 11]
+    qs, _, _ = oracle.qkv_proj(x, w, P, H, Hkv, d, rows=rows)
+    assert np.array_equal(qs, q[:, rows])
+    o = _bf((P, N, H // P, d), 9)
+    wo = _bf((hidden, H * d), 10)
+    seq = o.double().permute(1, 0, 2, 3).reshape(N, H * d)
+    np.testing.assert_allclose(oracle.out_proj(o, wo), (seq @ wo.double().T).numpy(), rtol=0, atol=1e-12)
