@@ -41,11 +41,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
-FWD_LAUNCHES = 4   # doc-bounds (3) + the attention kernel
-BWD_LAUNCHES = 8   # doc-bounds (5) + delta, dK/dV and dQ kernels
+FWD_LAUNCHES = 2   # doc-bounds + the attention kernel
+BWD_LAUNCHES = 4   # doc-bounds + delta, dK/dV and dQ kernels
 # Workloads the default run measures after the headline one, with the steps
 # each times (the million-token step lasts about a second: 3 are enough).
-SUB_WORKLOADS = ("tiny", "long131k", "million", "train")
+SUB_WORKLOADS = ("tiny", "long131k", "million", "train", "hybrid_kv2")
 SUB_STEPS = {"million": 3}
 
 
@@ -168,7 +168,7 @@ class Timer:
     def __init__(self, stream, enabled: bool):
         self.stream = stream
         self.enabled = enabled
-        self.ev = {"attn_fwd": [], "attn_bwd": [], "relayout": [], "exchange": []}
+        self.ev = {"attn_fwd": [], "attn_bwd": [], "relayout": [], "exchange": [], "merge": []}
 
     def __call__(self, kind, fn):
         if not self.enabled:
@@ -229,6 +229,24 @@ def build_single(U, w, inp, dev, timed, attn_ranks=None):
 
     launches = 3 + FWD_LAUNCHES * len(ranks) + 1 + ((1 + BWD_LAUNCHES * len(ranks) + 3) if w.backward else 0)
     return step, launches, ws
+
+
+def build_hybrid(U, w, inp, dev, timed):
+    """One GPU, the Ulysses x ring hybrid (fewer KV heads than ranks): the
+    U-way exchange of Q, K, V, each rank's ring steps as key-window passes of
+    the forward and their merge, the U-way exchange of O back. Returns (step,
+    our kernel launches per step, workspace)."""
+    from long_context_sequence_ulysses_b200 import hybrid
+    plan = hybrid.HybridPlan(w.N, w.H, w.Hkv, w.d, w.P, w.ulysses, dev)
+    pos = inp["position_ids"]
+    o_seq = torch.empty_like(inp["q"])
+    n_steps = sum(len(c) for _, c in plan.steps())
+    n_ranks = plan.U * plan.R
+
+    def step():
+        hybrid.forward(inp["q"], inp["k"], inp["v"], pos, w.P, w.ulysses, plan=plan, out=o_seq, timed=timed)
+
+    return step, 3 + FWD_LAUNCHES * n_steps + n_ranks + 1, plan.ws
 
 
 def build_fused(U, w, inp, dev):
@@ -346,7 +364,9 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     stream = torch.cuda.current_stream(dev)
     timed = Timer(stream, False)
     attn_ranks = [0] if w.name == "million" else None
-    if world == 1:
+    if world == 1 and w.ulysses:
+        step, launches_per_step, ws = build_hybrid(U, w, inp, dev, timed)
+    elif world == 1:
         step, launches_per_step, ws = build_single(U, w, inp, dev, timed, attn_ranks)
     else:
         step, launches_per_step, ws = build_multi(U, w, inp, dev, timed, world, rank, args.chunks)
@@ -391,6 +411,7 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     bwd_avg, bwd_sum = timed.stats("attn_bwd")
     _, rel_sum = timed.stats("relayout")
     _, exch_sum = timed.stats("exchange")
+    _, merge_sum = timed.stats("merge")
 
     # the whole job: all ranks (all GPUs), all heads of the ranks that ran
     total_flop = fwd_flop_step + bwd_flop_step
@@ -400,11 +421,14 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     long_step = ms_step > 500.0
     bf16_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
     peak_source = "%s %s" % (peak_kind, "sustained" if long_step else "burst")
-    launches_attn = w.P * world if world == 1 else world        # attention launches over the job, all ranks
-    fwd_flop_launch = fwd_flop / launches_attn
-    bwd_flop_launch = bwd_flop / launches_attn
-    achieved = fwd_flop_launch / (fwd_avg * 1e-3) / 1e12 if fwd_avg else None
-    bwd_ach = bwd_flop_launch / (bwd_avg * 1e-3) / 1e12 if bwd_avg else None
+    n_fwd = len(timed.ev["attn_fwd"]) // steps if timed.ev["attn_fwd"] else 1   # attention launches per step
+    n_bwd = len(timed.ev["attn_bwd"]) // steps if timed.ev["attn_bwd"] else 1
+    fwd_flop_launch = fwd_flop_step / n_fwd
+    bwd_flop_launch = bwd_flop_step / n_bwd
+    # the attention work of a step over the time its launches took (launches of
+    # equal size for Ulysses; the hybrid's ring steps differ in size)
+    achieved = fwd_flop_step / (fwd_sum / steps * 1e-3) / 1e12 if fwd_sum else None
+    bwd_ach = bwd_flop_step / (bwd_sum / steps * 1e-3) / 1e12 if bwd_sum else None
     traffic = lookup_traffic("attn_fwd_kernel", w.name) if world == 1 else None
 
     def roof(kernel, ach, flop_launch, traffic_b):
@@ -429,7 +453,10 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
         "config": {
             "workload": w.name, "N": w.N, "P": w.P if world == 1 else world, "H": w.H, "Hkv": w.Hkv, "d": w.d,
             "docs": w.docs, "documents": len(lengths), "unmasked_pairs": pairs, "backward": w.backward,
-            "step": (("seq_to_head(Q,K,V) for all P ranks; attn_fwd for "
+            "step": (("Ulysses x ring hybrid, U=%d x R=%d: seq_to_head(Q,K,V) over U; per rank its ring steps "
+                      "(key-window attention) and their merge; head_to_seq(O) over U"
+                      % (w.ulysses, w.P // w.ulysses)) if (w.ulysses and world == 1) else
+                     ("seq_to_head(Q,K,V) for all P ranks; attn_fwd for "
                       + ("rank 0's head slice" if attn_ranks else "each rank's head slice")
                       + ("; seq_to_head(dO), attn_bwd per rank, head_to_seq(dQ,dK,dV)" if w.backward else "")
                       + "; head_to_seq(O) for all ranks") if world == 1 else
@@ -443,8 +470,9 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
                   if w.N * w.H * w.d * 2 > (126 << 20) else
                   "inputs smaller than L2; each step re-reads them from L2 (launch-latency bound, no roofline claim)",
         },
-        "roofline": roof("attn_fwd_kernel (timed with the doc-bounds launch that precedes it)", achieved,
-                         fwd_flop_launch, traffic),
+        "roofline": roof("attn_fwd_kernel (timed with the doc-bounds launch that precedes it)"
+                         + ("; the hybrid's key-window passes, merges not included" if w.ulysses else ""),
+                         achieved, fwd_flop_launch, traffic),
         "attn_fwd_ms_per_launch": round(fwd_avg, 4) if fwd_avg else None,
         "attn_bwd_ms_per_launch": round(bwd_avg, 4) if bwd_avg else None,
         "attn_bwd_tflops": round(bwd_ach, 2) if bwd_ach else None,
@@ -463,6 +491,8 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
                            "frac_of_spec_8000": round(rb / SPEC_HBM_GBS, 4)}
     if exch_sum:
         out["exchange_ms_per_step"] = round(exch_sum / steps, 4)
+    if merge_sum:
+        out["merge_ms_per_step"] = round(merge_sum / steps, 4)
     if world > 1:
         # device memory one step allocates beyond what is resident before it
         # (exchange buffers and head slices; smaller with more head chunks)
@@ -478,13 +508,97 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
         out["chunks"] = args.chunks
     if headline:
         out["e2e"] = run_e2e(U, w, inp, args, dev) if (args.e2e_steps > 0 and world == 1) else None
-    if world == 1 and args.fused and not attn_ranks:
+    if world == 1 and args.fused and not attn_ranks and not w.ulysses:
         out["fused_step"] = time_fused(U, w, inp, dev, steps, total_flop)
     if headline and rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, inp, args)
     del inp, step, ws
     torch.cuda.empty_cache()
     return out
+
+
+def measure_layer(U, w, dev, args, steps, warmup):
+    """The layer step around the path on one GPU, all P ranks: the QKV
+    projection written straight into every rank's head slice (projection and
+    first exchange in one kernel), the attention of each rank, and the output
+    projection read straight from the head slices (second exchange and
+    projection in one kernel). Synthetic activations and random-init weights
+    of the workload's shape (hidden = H*d)."""
+    from workloads import projection_inputs
+    inp = make_inputs(w, device=dev)
+    pin = projection_inputs(w, device=dev)
+    pairs, fwd_flop, _, _ = workload_work(w, inp["lengths"])
+    hidden = w.H * w.d
+    qkv_flop = 2.0 * w.N * hidden * (w.H + 2 * w.Hkv) * w.d
+    out_flop = 2.0 * w.N * (w.H * w.d) * hidden
+    P, N, d, Hl, Hkvl = w.P, w.N, w.d, w.Hl, w.Hkvl
+    q_all = torch.empty((P, N, Hl, d), dtype=torch.bfloat16, device=dev)
+    k_all = torch.empty((P, N, Hkvl, d), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty_like(k_all)
+    o_all = torch.empty_like(q_all)
+    lse_all = torch.empty((w.H, N), dtype=torch.float32, device=dev)
+    y = torch.empty((N, hidden), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(U.workspace_bytes(N, Hl, Hkvl, d, False), dtype=torch.uint8, device=dev)
+    pws = U.proj_workspace(dev)
+    pos = inp["position_ids"]
+    stream = torch.cuda.current_stream(dev)
+    timed = Timer(stream, False)
+    timed.ev["gemm_qkv"], timed.ev["gemm_out"] = [], []
+
+    def step():
+        timed("gemm_qkv", lambda: U.qkv_proj(pin["x"], pin["w_qkv"], P, w.H, w.Hkv, d, q_out=q_all, k_out=k_all,
+                                             v_out=v_all, ws=pws))
+        for r in range(P):
+            timed("attn_fwd", lambda: U.attn_fwd(q_all[r], k_all[r], v_all[r], pos, out=o_all[r],
+                                                 lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws))
+        timed("gemm_out", lambda: U.out_proj(o_all, pin["w_o"], out=y, ws=pws))
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    U.sync_status(ws)
+    U.sync_status(pws)
+    timed.enabled = args.kernel_events
+    sampler = ClockSampler(int(str(dev).split(":")[-1]) if ":" in str(dev) else 0)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    U.sync_status(ws)
+    U.sync_status(pws)
+    ms = t0.elapsed_time(t1) / steps
+    peaks, peak_kind = load_peaks()
+    peak = peaks["bf16_tflops"]
+    total = fwd_flop + qkv_flop + out_flop
+    rec = {"value": round(total / (ms * 1e-3) / 1e12, 2), "ms_per_step": round(ms, 4), "steps": steps,
+           "warmup": warmup, "config": {"workload": w.name + "_layer", "N": N, "P": P, "H": w.H, "Hkv": w.Hkv,
+                                        "d": d, "hidden": hidden, "step_flop": total,
+                                        "step": "qkv_proj into every rank's head slice (fused first exchange); "
+                                                "attn_fwd per rank; out_proj from the head slices (fused second "
+                                                "exchange)", "weights": "random-init, N(0, 1/hidden), seeded"},
+           "clocks": clocks, "gpu_launches": (2 + FWD_LAUNCHES * P) * steps}
+    for kind, flop, name in (("gemm_qkv", qkv_flop, "qkv_proj (proj_gemm_kernel<256>)"),
+                             ("gemm_out", out_flop, "out_proj (proj_gemm_kernel<256>)")):
+        avg, _ = timed.stats(kind)
+        if avg:
+            ach = flop / (avg * 1e-3) / 1e12
+            rec["roofline_" + kind] = {"kernel": name, "bound": "tensor", "achieved": round(ach, 2), "peak": peak,
+                                       "peak_source": peak_kind + " burst", "unit": "TFLOP/s",
+                                       "frac": round(ach / peak, 4), "frac_of_spec_2250": round(ach / SPEC_BF16_TFLOPS, 4),
+                                       "flop_per_launch": flop, "ms_per_launch": round(avg, 4), "traffic": None}
+    fwd_avg, fwd_sum = timed.stats("attn_fwd")
+    if fwd_sum:
+        rec["attn_fwd_tflops"] = round(fwd_flop / (fwd_sum / steps * 1e-3) / 1e12, 2)
+    del inp, pin, q_all, k_all, v_all, o_all, y
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_gpu(args):
@@ -512,6 +626,7 @@ def run_gpu(args):
             for key in ("metric", "unit", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "dtype", "data"):
                 r.pop(key, None)
             subs[sub] = r
+        subs["llama8b_layer"] = measure_layer(U, WORKLOADS["llama8b"], dev, args, args.steps, max(3, args.warmup))
         out["workloads"] = subs
         out["gpu_launches"] += sum(r["gpu_launches"] for r in subs.values())
     if dist is not None:

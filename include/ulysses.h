@@ -83,6 +83,20 @@ int ulysses_head_to_seq(const void *src, void *dst, int64_t N, int P, int Hx, in
                         int rank, void *stream);
 
 /*
+ * The same two exchanges for a slice of heads: the sequence-side rows hold
+ * row_heads heads ([P][N/P][row_heads][d]), of which heads [head0, head0+Hx)
+ * are exchanged, read from (seq_to_head) or written into (head_to_seq) those
+ * rows in place; the head side is as above for Hx heads. This is the exchange
+ * of one chunk of heads of the head-chunked variant (page "Ulysses 序列並行：百萬
+ * Token 上下文訓練", section "競品分析", UPipe), with no copy of the chunk.
+ * Requires head0 >= 0 and head0 + Hx <= row_heads, plus the conditions above.
+ */
+int ulysses_seq_to_head_heads(const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
+                              int row_heads, int head0, void *stream);
+int ulysses_head_to_seq_heads(const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
+                              int row_heads, int head0, void *stream);
+
+/*
  * Bytes of device workspace that ulysses_attn_fwd (backward = 0) or
  * ulysses_attn_bwd (backward = 1) need for these sizes. The workspace holds
  * the per-token document starts, per-tile key ranges, the tile schedule, the
@@ -122,6 +136,43 @@ int ulysses_attn_fwd_fused(const void *q_seq, const void *k_seq, const void *v_s
                            const int32_t *position_ids, int64_t N, int P, int H, int Hkv,
                            int d, int rank, float scale, void *o_seq, float *lse,
                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One ring step of the Ulysses x ring hybrid (for Hkv < P, where Ulysses
+ * alone runs out of heads: page "Ulysses 序列並行：百萬 Token 上下文訓練",
+ * section "競品分析"; page "Ulysses verteilt Millionen-Token-Kontexte auf
+ * mehrere GPUs", section "Wann Ulysses sinnvoll ist"): the attention of the
+ * query rows [q_lo, q_hi) over the keys [kv_lo, kv_hi) only -- the chunk of
+ * keys and values a rank holds at that step of the ring.
+ *
+ *   q [N][Hl][d], k, v [N][Hkvl][d], position_ids [N]: as ulysses_attn_fwd
+ *         (whole-sequence indices; only the rows and keys of the windows are read).
+ *   o     [q_hi - q_lo][Hl][d] bf16: row i - q_lo is the partial output of row i,
+ *         normalised over the keys it sees in the window.
+ *   lse   [Hl][q_hi - q_lo] fp32: natural-log sum of exp over those keys.
+ * Row i sees keys j with max(doc_start(i), kv_lo) <= j <= min(i, kv_hi - 1); a
+ * row that sees none gets o = 0 and lse = -inf. Requires 0 <= q_lo <= q_hi <= N
+ * and 0 <= kv_lo <= kv_hi <= N (ULYSSES_ERR_INVALID otherwise). The workspace
+ * is the forward one for (N, Hl). Partials of disjoint windows combine with
+ * ulysses_attn_merge into the attention over their union.
+ */
+int ulysses_attn_fwd_window(const void *q, const void *k, const void *v, const int32_t *position_ids,
+                            int64_t N, int Hl, int Hkvl, int d, int64_t q_lo, int64_t q_hi, int64_t kv_lo,
+                            int64_t kv_hi, float scale, void *o, float *lse, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
+ * Merge of R partial attention results over disjoint key sets (the ring
+ * steps of one rank) into the result over their union:
+ *   L = log sum_s exp(lse_s),  o = sum_s exp(lse_s - L) o_s,  lse = L.
+ *   o_parts   [R][M][Hl][d] bf16, lse_parts [R][Hl][M] fp32 (lse_s = -inf: no key).
+ *   o         [M][Hl][d] bf16 (rounded once), lse [Hl][lse_ld] fp32 (first M
+ *             columns of each row written); a row with no key in any part
+ *             gets o = 0, lse = -inf.
+ * Requires 1 <= R <= 64 and lse_ld >= M. Accumulates in fp32.
+ */
+int ulysses_attn_merge(const void *o_parts, const float *lse_parts, int R, int64_t M, int Hl, int d, void *o,
+                       float *lse, int64_t lse_ld, void *stream);
 
 /*
  * Attention backward for one rank's head slice: gradients of sum(dout * o).
@@ -177,6 +228,47 @@ int ulysses_attn_bwd_fused(const void *q_seq, const void *k_seq, const void *v_s
 int ulysses_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                              const int32_t *position_ids, int64_t N, int Hl, int Hkvl, int d,
                              float scale, void *o, float *lse, void *stream);
+
+/*
+ * The projections on either side of the exchange, with the exchange fused in
+ * (page "Hugging Face并行加速：10倍提升超长序列训练效率", section
+ * "Ulysses的工作原理", steps QKV投影 and 输出投影; page "DeepSpeed Ulysses 详解",
+ * section "DeepSpeed-Ulysses 的核心机制", items 2 and 6). Every rank projects its
+ * own tokens with the full weights; here the tokens of all P ranks are
+ * projected by one tensor-core GEMM (bf16 operands, fp32 accumulation, bf16
+ * results rounded once). The workspace is ulysses_proj_workspace_bytes()
+ * bytes of device memory (a status word; bounded device waits report there,
+ * read by ulysses_sync_status).
+ */
+size_t ulysses_proj_workspace_bytes(void);
+
+/*
+ * QKV projection fused with the first exchange:
+ *   x      [N][hidden] bf16: the P sequence shards ([P][N/P][hidden]).
+ *   w_qkv  [(H+2Hkv)*d][hidden] bf16: output column c = x . w_qkv[c]; columns
+ *          [0, H*d) are Q's heads, then K's, then V's, d per head.
+ *   q_heads [P][N][H/P][d], k_heads, v_heads [P][N][Hkv/P][d]: every rank's
+ *          head slice (the layout ulysses_seq_to_head produces): head g of token
+ *          n lands in rank g/(heads/P), slot g%(heads/P).
+ * Requires H % P == Hkv % P == 0, N % P == 0, d in {32,64,128}, hidden a
+ * positive multiple of 64 and (H+2Hkv)*d a multiple of 128
+ * (ULYSSES_ERR_UNSUPPORTED otherwise).
+ */
+int ulysses_qkv_proj(const void *x, const void *w_qkv, int64_t N, int hidden, int P, int H, int Hkv, int d,
+                     void *q_heads, void *k_heads, void *v_heads, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Output projection fused with the second exchange:
+ *   o_heads [P][N][H/P][d] bf16: every rank's head slice of the attention
+ *           output; read in the sequence order of heads (global head
+ *           r*H/P + h at columns ((r*H/P + h)*d ...) of a token's row).
+ *   w_o     [hidden][H*d] bf16.
+ *   y       [N][hidden] bf16: y[n] = o_seq[n] . w_o^T.
+ * Requires H % P == 0, N % P == 0, d in {64,128} (ULYSSES_ERR_UNSUPPORTED for
+ * d = 32) and hidden a multiple of 128.
+ */
+int ulysses_out_proj(const void *o_heads, const void *w_o, int64_t N, int hidden, int P, int H, int d, void *y,
+                     void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Synchronise `stream` and report the status the latest attention call left

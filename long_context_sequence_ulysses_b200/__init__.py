@@ -25,8 +25,9 @@ import torch
 
 __all__ = [
     "UlyssesError", "library_path", "seq_to_head", "head_to_seq", "workspace_bytes", "attn_fwd",
-    "attn_fwd_fused", "attn_bwd", "attn_bwd_fused", "sync_status", "set_wait_limit_ns", "set_debug_flags",
-    "version",
+    "attn_fwd_fused", "attn_bwd", "attn_bwd_fused", "attn_fwd_window", "attn_merge", "qkv_proj",
+    "out_proj", "proj_workspace", "sync_status",
+    "set_wait_limit_ns", "set_debug_flags", "version",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -57,6 +58,8 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_version.restype = ctypes.c_char_p
     lib.ulysses_seq_to_head.argtypes = [P, P, I64, I32, I32, I32, I32, P]
     lib.ulysses_head_to_seq.argtypes = [P, P, I64, I32, I32, I32, I32, P]
+    lib.ulysses_seq_to_head_heads.argtypes = [P, P, I64, I32, I32, I32, I32, I32, I32, P]
+    lib.ulysses_head_to_seq_heads.argtypes = [P, P, I64, I32, I32, I32, I32, I32, I32, P]
     lib.ulysses_attn_workspace_bytes.argtypes = [I64, I32, I32, I32, I32]
     lib.ulysses_attn_workspace_bytes.restype = SZ
     lib.ulysses_attn_fwd.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, SZ, P]
@@ -64,13 +67,22 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_attn_bwd.argtypes = [P, P, P, P, P, P, P, I64, I32, I32, I32, F32, P, P, P, P, SZ, P]
     lib.ulysses_attn_bwd_fused.argtypes = [P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, F32, P, P, P, P, SZ,
                                            P]
+    lib.ulysses_attn_fwd_window.argtypes = [P, P, P, P, I64, I32, I32, I32, I64, I64, I64, I64, F32, P, P, P, SZ,
+                                            P]
+    lib.ulysses_attn_merge.argtypes = [P, P, I32, I64, I32, I32, P, P, I64, P]
+    lib.ulysses_proj_workspace_bytes.argtypes = []
+    lib.ulysses_proj_workspace_bytes.restype = SZ
+    lib.ulysses_qkv_proj.argtypes = [P, P, I64, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]
+    lib.ulysses_out_proj.argtypes = [P, P, I64, I32, I32, I32, I32, P, P, SZ, P]
     lib.ulysses_sync_status.argtypes = [P, P]
     lib.ulysses_set_wait_limit_ns.argtypes = [I64]
     lib.ulysses_set_wait_limit_ns.restype = None
     lib.ulysses_set_debug_flags.argtypes = [ctypes.c_uint32]
     lib.ulysses_set_debug_flags.restype = None
-    for name in ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_fwd_fused",
-                 "ulysses_attn_bwd", "ulysses_attn_bwd_fused", "ulysses_sync_status"):
+    for name in ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_seq_to_head_heads",
+                 "ulysses_head_to_seq_heads", "ulysses_attn_fwd", "ulysses_attn_fwd_fused",
+                 "ulysses_attn_bwd", "ulysses_attn_bwd_fused", "ulysses_attn_fwd_window", "ulysses_attn_merge",
+                 "ulysses_qkv_proj", "ulysses_out_proj", "ulysses_sync_status"):
         getattr(lib, name).restype = I32
     return lib
 
@@ -148,11 +160,16 @@ def _pos32(pos: torch.Tensor, N: int) -> torch.Tensor:
     return pos.contiguous()
 
 
-def seq_to_head(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+def seq_to_head(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None,
+                heads: Optional[Tuple[int, int]] = None) -> torch.Tensor:
     """[N][Hx][d] (= P rank buffers [P][N/P][Hx][d]) -> [P][N][Hx/P][d], or
-    rank r's slice [N][Hx/P][d] when ``rank >= 0``."""
-    N, Hx, d = _dims("src", src, 3)
-    _spec("src", src, (N, Hx, d))
+    rank r's slice [N][Hx/P][d] when ``rank >= 0``. With ``heads=(head0, n)``
+    only heads [head0, head0+n) of src's rows are exchanged (read in place)."""
+    N, row_heads, d = _dims("src", src, 3)
+    _spec("src", src, (N, row_heads, d))
+    head0, Hx = (0, row_heads) if heads is None else (int(heads[0]), int(heads[1]))
+    if head0 < 0 or Hx < 1 or head0 + Hx > row_heads:
+        raise ValueError(f"heads [{head0}, {head0 + Hx}) outside the {row_heads} heads of src")
     if P < 1 or Hx % P:
         raise ValueError(f"head count {Hx} must be divisible by P={P}")
     shape = (P, N, Hx // P, d) if rank < 0 else (N, Hx // P, d)
@@ -162,13 +179,20 @@ def seq_to_head(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.T
     else:
         _same_cuda(("src", src))
         out = torch.empty(shape, dtype=src.dtype, device=src.device)
-    _check(_lib.ulysses_seq_to_head(_ptr(src), _ptr(out), N, P, Hx, d, rank, _stream(src)))
+    if heads is None:
+        _check(_lib.ulysses_seq_to_head(_ptr(src), _ptr(out), N, P, Hx, d, rank, _stream(src)))
+    else:
+        _check(_lib.ulysses_seq_to_head_heads(_ptr(src), _ptr(out), N, P, Hx, d, rank, row_heads, head0,
+                                              _stream(src)))
     return out
 
 
-def head_to_seq(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+def head_to_seq(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.Tensor] = None,
+                head0: Optional[int] = None) -> torch.Tensor:
     """[P][N][Hx/P][d] -> [N][Hx][d]; with ``rank >= 0`` src is rank r's slice
-    [N][Hx/P][d] and only its heads of ``out`` are written."""
+    [N][Hx/P][d] and only its heads of ``out`` are written. With ``head0`` the
+    result goes to heads [head0, head0+Hx) of ``out`` [N][row_heads][d] (the
+    other heads are kept)."""
     if rank < 0:
         Pp, N, Hl, d = _dims("src", src, 4)
         if Pp != P:
@@ -178,6 +202,17 @@ def head_to_seq(src: torch.Tensor, P: int, rank: int = -1, out: Optional[torch.T
         N, Hl, d = _dims("src", src, 3)
         _spec("src", src, (N, Hl, d))
     Hx = Hl * P
+    if head0 is not None:
+        if out is None:
+            raise ValueError("head_to_seq with head0 needs `out`")
+        row_heads = _dims("out", out, 3)[1]
+        if head0 < 0 or head0 + Hx > row_heads:
+            raise ValueError(f"heads [{head0}, {head0 + Hx}) outside the {row_heads} heads of out")
+        _spec("out", out, (N, row_heads, d))
+        _same_cuda(("src", src), ("out", out))
+        _check(_lib.ulysses_head_to_seq_heads(_ptr(src), _ptr(out), N, P, Hx, d, rank, row_heads, int(head0),
+                                              _stream(src)))
+        return out
     shape = (N, Hx, d)
     if out is not None:
         _spec("out", out, shape)
@@ -245,6 +280,122 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position_ids: to
     _check(_lib.ulysses_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), N, Hl, Hkvl, d, sc, _ptr(out), _ptr(lse),
                                  _ptr(ws), ws.numel(), _stream(q)))
     return out, lse
+
+
+def attn_fwd_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position_ids: torch.Tensor,
+                    q_lo: int, q_hi: int, kv_lo: int, kv_hi: int, scale: Optional[float] = None,
+                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One ring step: the attention of rows [q_lo, q_hi) of the head slice
+    q [N][Hl][d] over the keys [kv_lo, kv_hi) of k/v [N][Hkvl][d] only.
+    Returns (o [q_hi-q_lo][Hl][d] bf16, lse [Hl][q_hi-q_lo] fp32); rows that
+    see no key get o = 0, lse = -inf."""
+    N, Hl, d = _dims("q", q, 3)
+    Hkvl = _dims("k", k, 3)[1]
+    _spec("q", q, (N, Hl, d))
+    _spec("k", k, (N, Hkvl, d))
+    _spec("v", v, (N, Hkvl, d))
+    _heads_ok(Hl, Hkvl)
+    if not (0 <= q_lo <= q_hi <= N and 0 <= kv_lo <= kv_hi <= N):
+        raise ValueError(f"windows [{q_lo}, {q_hi}) and [{kv_lo}, {kv_hi}) must lie in [0, {N}]")
+    M = q_hi - q_lo
+    if out is not None:
+        _spec("out", out, (M, Hl, d))
+    if lse is not None:
+        _spec("lse", lse, (Hl, M), torch.float32)
+    pos = _pos32(position_ids, N)
+    _same_cuda(("q", q), ("k", k), ("v", v), ("position_ids", pos), *((("out", out),) if out is not None else ()),
+               *((("lse", lse),) if lse is not None else ()))
+    if out is None:
+        out = torch.empty((M, Hl, d), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((Hl, M), dtype=torch.float32, device=q.device)
+    ws = _workspace(ws, workspace_bytes(N, Hl, Hkvl, d, False), q.device)
+    sc = 0.0 if scale is None else float(scale)
+    _check(_lib.ulysses_attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), N, Hl, Hkvl, d, int(q_lo), int(q_hi),
+                                        int(kv_lo), int(kv_hi), sc, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                        _stream(q)))
+    return out, lse
+
+
+def attn_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Merge R partial results over disjoint key sets: o_parts [R][M][Hl][d]
+    bf16, lse_parts [R][Hl][M] fp32 -> (o [M][Hl][d], lse [Hl][M]). ``lse`` may
+    be a column slice of a wider [Hl][*] fp32 tensor (rows contiguous)."""
+    R, M, Hl, d = _dims("o_parts", o_parts, 4)
+    _spec("o_parts", o_parts, (R, M, Hl, d))
+    _spec("lse_parts", lse_parts, (R, Hl, M), torch.float32)
+    if out is not None:
+        _spec("out", out, (M, Hl, d))
+    ld = M
+    if lse is not None:
+        if not isinstance(lse, torch.Tensor) or lse.dtype != torch.float32 or tuple(lse.shape) != (Hl, M) \
+                or lse.stride(1) != 1 or (Hl > 1 and lse.stride(0) < M):
+            raise ValueError(f"lse must be fp32 [{Hl}][{M}] with contiguous rows")
+        ld = lse.stride(0) if Hl > 1 else M
+    _same_cuda(("o_parts", o_parts), ("lse_parts", lse_parts), *((("out", out),) if out is not None else ()),
+               *((("lse", lse),) if lse is not None else ()))
+    if out is None:
+        out = torch.empty((M, Hl, d), dtype=o_parts.dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((Hl, M), dtype=torch.float32, device=o_parts.device)
+    _check(_lib.ulysses_attn_merge(_ptr(o_parts), _ptr(lse_parts), R, M, Hl, d, _ptr(out), _ptr(lse), ld,
+                                   _stream(o_parts)))
+    return out, lse
+
+
+def proj_workspace(device) -> torch.Tensor:
+    """Workspace of the projection calls (a status word)."""
+    return torch.zeros(int(_lib.ulysses_proj_workspace_bytes()), dtype=torch.uint8, device=device)
+
+
+def qkv_proj(x: torch.Tensor, w_qkv: torch.Tensor, P: int, H: int, Hkv: int, d: int,
+             q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None,
+             v_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
+             ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """QKV projection of the P sequence shards x [N][hidden] with w_qkv
+    [(H+2Hkv)*d][hidden], written straight into every rank's head slice:
+    returns q [P][N][H/P][d], k and v [P][N][Hkv/P][d]."""
+    N, hidden = _dims("x", x, 2)
+    _spec("x", x, (N, hidden))
+    _spec("w_qkv", w_qkv, ((H + 2 * Hkv) * d, hidden))
+    if P < 1 or H % P or Hkv % P:
+        raise ValueError(f"H={H} and Hkv={Hkv} must be divisible by P={P}")
+    shapes = ((P, N, H // P, d), (P, N, Hkv // P, d), (P, N, Hkv // P, d))
+    outs = []
+    for name, t, shp in (("q_out", q_out, shapes[0]), ("k_out", k_out, shapes[1]), ("v_out", v_out, shapes[2])):
+        if t is not None:
+            _spec(name, t, shp)
+        outs.append(t)
+    _same_cuda(("x", x), ("w_qkv", w_qkv), *((n, t) for n, t in zip(("q_out", "k_out", "v_out"), outs)
+                                             if t is not None))
+    outs = [torch.empty(shp, dtype=torch.bfloat16, device=x.device) if t is None else t
+            for t, shp in zip(outs, shapes)]
+    ws = proj_workspace(x.device) if ws is None else ws
+    _check(_lib.ulysses_qkv_proj(_ptr(x), _ptr(w_qkv), N, hidden, P, H, Hkv, d, _ptr(outs[0]), _ptr(outs[1]),
+                                 _ptr(outs[2]), _ptr(ws), ws.numel(), _stream(x)))
+    return tuple(outs)
+
+
+def out_proj(o_heads: torch.Tensor, w_o: torch.Tensor, out: Optional[torch.Tensor] = None,
+             ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Output projection read straight from every rank's head slice of the
+    attention output o_heads [P][N][H/P][d], with w_o [hidden][H*d]:
+    returns y [N][hidden] in the sequence layout."""
+    P, N, Hl, d = _dims("o_heads", o_heads, 4)
+    _spec("o_heads", o_heads, (P, N, Hl, d))
+    hidden = _dims("w_o", w_o, 2)[0]
+    _spec("w_o", w_o, (hidden, P * Hl * d))
+    if out is not None:
+        _spec("out", out, (N, hidden))
+    _same_cuda(("o_heads", o_heads), ("w_o", w_o), *((("out", out),) if out is not None else ()))
+    if out is None:
+        out = torch.empty((N, hidden), dtype=torch.bfloat16, device=o_heads.device)
+    ws = proj_workspace(o_heads.device) if ws is None else ws
+    _check(_lib.ulysses_out_proj(_ptr(o_heads), _ptr(w_o), N, hidden, P, P * Hl, d, _ptr(out), _ptr(ws), ws.numel(),
+                                 _stream(o_heads)))
+    return out
 
 
 def _rank_heads(H: int, Hkv: int, P: int, rank: int) -> Tuple[int, int]:

@@ -13,8 +13,10 @@
 //
 // Three kernels, all deterministic (no atomics):
 //  1. prep: D_i and -LSE_i*log2(e) per (head, row) into a 128-padded layout.
-//  2. dK/dV: one CTA per (key tile, KV head) loops over the query heads of the
-//     GQA group and the query tiles that see the key tile:
+//  2. dK/dV: one CTA per (key tile, KV head) loops over the query tiles that
+//     see the key tile and, for each, the query heads of the GQA group (heads
+//     inner: CTAs of neighbouring key tiles then read the same Q / dO tiles a
+//     few steps apart, while they are still in L2):
 //       S^T = K Q^T, dP^T = V dO^T       (SS MMA, M = keys, N = queries)
 //       P^T, dS^T -> bf16 into the first 64 columns of S^T / dP^T in TMEM
 //       dV += P^T dO, dK += dS^T Q      (TS MMA, dO / Q read MN-major)
@@ -266,8 +268,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
             for (int it = 0; it < n_it; ++it) {
                 const int s = it % C::NST, u = it / C::NST;
-                const int h = kvh * G + it / n_q;
-                const int qt = qt0 + it % n_q;
+                const int h = kvh * G + it % G;
+                const int qt = qt0 + it / G;
                 if (u > 0 && !mbar_wait(&qdo_empty[s], (u - 1) & 1, wc)) break;
                 mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES + 2 * 512);
                 tma_tile<D>(&tmQ, sQ + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int s = it % C::NST, u = it / C::NST;
-            const int q0 = (qt0 + it % n_q) * kTileM + part * kPartCols;   // first query of this part
+            const int q0 = (qt0 + it / G) * kTileM + part * kPartCols;   // first query of this part
             // warp-uniform waits: the tcgen05.ld below needs the whole warp converged
             if (!mbar_wait_warp(s_full, it & 1, wc)) { ok = false; break; }
             if (!mbar_wait_warp(&qdo_full[s], u & 1, wc)) { ok = false; break; }
@@ -370,8 +372,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const bool any_mask = __any_sync(0xffffffffu, (q0 < j) || (q0 + kPartCols - 1 >= dend));
             // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns;
             // the per-query values are fetched as float4 before waiting for the tensor-memory load
-            uint32_t pp[kPartCols / 2];
+            float pf[kPartCols];   // P^T in fp32: dS is formed from it, rounded once
             {
+                uint32_t pp[kPartCols / 2];
                 uint32_t sr[kPartCols];
                 tmem_ld32(tbase + C::T_S + lane_off + col, sr);
                 float4 nl[kPartCols / 4];
@@ -389,14 +392,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         if (qi < j || qi >= dend) x0 = -CUDART_INF_F;
                         if (qi + 1 < j || qi + 1 >= dend) x1 = -CUDART_INF_F;
                     }
-                    pp[e] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+                    pf[2 * e] = ex2_approx(x0);
+                    pf[2 * e + 1] = ex2_approx(x1);
+                    pp[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
                 }
+                tmem_st16(tbase + C::T_S + lane_off + col, pp);   // P^T (queries packed in pairs)
             }
-            tmem_st16(tbase + C::T_S + lane_off + col, pp);   // P^T (queries packed in pairs)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_ready);
-            // phase 2: dS^T = P^T (dP^T - D) from the bf16 P^T, bf16 into dP^T's columns
+            // phase 2: dS^T = P^T (dP^T - D) from the fp32 P^T, bf16 into dP^T's columns
             if (!mbar_wait_warp(dp_full, it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
@@ -411,10 +416,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int e = 0; e < kPartCols / 2; ++e) {
                     const float4 &d4 = dl[e >> 1];
                     const float b0 = (e & 1) ? d4.z : d4.x, b1 = (e & 1) ? d4.w : d4.y;
-                    const uint32_t pe = pp[e];
                     float t0, t1, d0, d1;
                     sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), b0, b1);
-                    mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
+                    mul2(d0, d1, pf[2 * e], pf[2 * e + 1], t0, t1);
                     dd[e] = pack_bf16x2(d0, d1);
                 }
                 tmem_st16(tbase + C::T_DP + lane_off + col, dd);   // dS^T
@@ -631,8 +635,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             const bool any_mask = __any_sync(0xffffffffu, (c0 < lo) || (c0 + kPartCols - 1 > i));
             // phase 1 (while dP(j) may still be computing): P = exp2(S * scale*log2(e)
-            // - LSE*log2(e)), kept as bf16 pairs
-            uint32_t pp[kPartCols / 2];
+            // - LSE*log2(e)), kept in fp32 so that dS is rounded only once
+            float pf[kPartCols];
             {
                 uint32_t sr[kPartCols];
                 tmem_ld32(tS, sr);
@@ -646,10 +650,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         if (key < lo || key > i) x0 = -CUDART_INF_F;
                         if (key + 1 < lo || key + 1 > i) x1 = -CUDART_INF_F;
                     }
-                    pp[e] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+                    pf[2 * e] = ex2_approx(x0);
+                    pf[2 * e + 1] = ex2_approx(x1);
                 }
             }
-            // phase 2: dS = P (dP - D) from the bf16 P, bf16 into S's columns
+            // phase 2: dS = P (dP - D) from the fp32 P, bf16 into S's columns
             if (!mbar_wait_warp(dp_full, j & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
@@ -659,10 +664,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 uint32_t dd[kPartCols / 2];
 #pragma unroll
                 for (int e = 0; e < kPartCols / 2; ++e) {
-                    const uint32_t pe = pp[e];
                     float t0, t1, d0, d1;
                     sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), di, di);
-                    mul2(d0, d1, __uint_as_float(pe << 16), __uint_as_float(pe & 0xffff0000u), t0, t1);
+                    mul2(d0, d1, pf[2 * e], pf[2 * e + 1], t0, t1);
                     dd[e] = pack_bf16x2(d0, d1);
                 }
                 tmem_st16(tS, dd);   // dS (keys packed in pairs)

@@ -82,9 +82,15 @@ struct FwdParams {
     __nv_bfloat16 *o;
     int64_t o_row_elems;   // elements between consecutive token rows of O
     int o_head0;
-    float *lse;
-    int N, T, Hl, Hkvl;
+    float *lse;            // [Hl][lse_ld]
+    int N, Hl, Hkvl;
     int q_head0, kv_head0;
+    // Query window: rows [q_lo, q_end) in query tiles q_tile0 .. q_tile0+T-1;
+    // O row i goes to o + (i - q_lo) * o_row_elems, its LSE to lse[h][i - q_lo].
+    int q_tile0, T, q_lo, q_end, lse_ld;
+    // Key window [kv_lo, kv_hi), key tiles kvlo_t .. kvhi_t (a ring step's
+    // chunk of keys; the whole sequence otherwise).
+    int kv_lo, kv_hi, kvlo_t, kvhi_t;
     float scale_log2;      // softmax scale * log2(e)
     int pair_heads;        // 1: items pair heads (T x Hl/2 items); 0: items pair tiles (ceil(T/2) x Hl)
     int items;
@@ -97,6 +103,8 @@ constexpr int kItemInts = 12;   // ints of one FwdItem
 
 // One work item. Head pairs: tile q_order[idx / (Hl/2)] of heads 2g, 2g+1,
 // g = idx % (Hl/2). Tile pairs: the pair q_order[idx / Hl] of head idx % Hl.
+// A tile's key tiles are those of its rows' documents inside the key window;
+// a tile with none (nA or nB == 0) only writes O = 0, LSE = -inf.
 struct FwdItem {
     int idx;       // work item index, -1: no more work
     int hA, hB, kvh, tA, tB;
@@ -121,23 +129,33 @@ __device__ __forceinline__ FwdItem decode_item(const FwdParams &p, int idx)
         it.kvh = it.hA / (p.Hl / p.Hkvl);
         it.tA = it.tB = t;
         it.hasB = 1;
-        it.j0 = p.tile_lo[t] / kTileN;
-        it.nA = it.nB = it.n_union = t - it.j0 + 1;
+        it.j0 = max(p.tile_lo[t] / kTileN, p.kvlo_t);
+        it.nA = it.nB = it.n_union = max(0, min(t, p.kvhi_t) - it.j0 + 1);
         it.bstart = 0;
         return it;
     }
     const int pair = p.q_order[idx / p.Hl];
     it.hA = it.hB = idx % p.Hl;
     it.kvh = it.hA / (p.Hl / p.Hkvl);
-    it.tA = 2 * pair;
-    it.tB = 2 * pair + 1;
-    it.hasB = it.tB < p.T ? 1 : 0;
-    it.j0 = p.tile_lo[it.tA] / kTileN;
-    it.nA = it.tA - it.j0 + 1;
-    const int loB = it.hasB ? p.tile_lo[it.tB] / kTileN : 0;
-    it.bstart = it.hasB ? loB - it.j0 : 0;
-    it.nB = it.hasB ? it.tB - loB + 1 : 0;
-    it.n_union = it.hasB ? it.tB - it.j0 + 1 : it.nA;
+    it.tA = p.q_tile0 + 2 * pair;
+    it.tB = it.tA + 1;
+    it.hasB = it.tB < p.q_tile0 + p.T ? 1 : 0;
+    const int loA = max(p.tile_lo[it.tA] / kTileN, p.kvlo_t);
+    const int hiA = min(it.tA, p.kvhi_t);
+    it.nA = max(0, hiA - loA + 1);
+    const int loB = it.hasB ? max(p.tile_lo[it.tB] / kTileN, p.kvlo_t) : 0;
+    const int hiB = min(it.tB, p.kvhi_t);
+    it.nB = it.hasB ? max(0, hiB - loB + 1) : 0;
+    // B's range starts no earlier than A's and ends no earlier, with no gap
+    if (it.nA > 0) {
+        it.j0 = loA;
+        it.bstart = it.nB > 0 ? loB - loA : 0;
+        it.n_union = it.nB > 0 ? hiB - loA + 1 : it.nA;
+    } else {
+        it.j0 = it.nB > 0 ? loB : 0;
+        it.bstart = 0;
+        it.n_union = it.nB;
+    }
     return it;
 }
 
@@ -228,6 +246,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_holder;
+    // Launched as a programmatic dependent of the doc-bounds kernel: everything
+    // above overlapped it; the schedule, the document starts and the status
+    // word it writes are read only from here on.
+    griddep_wait();
 
     // A CTA that starts after another one has timed out skips its work.
     WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
@@ -282,7 +304,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     ++qcount[x];
                     return true;
                 };
-                bool ok = load_q(0);
+                bool ok = w.nA > 0 ? load_q(0) : true;
                 for (int j = 0; ok && j < w.n_union; ++j, ++kcount) {
                     const int s = kcount % C::KST, u = kcount / C::KST;
                     if (u > 0 && !mbar_wait(&k_empty[s], (u - 1) & 1, wc)) { ok = false; break; }
@@ -292,7 +314,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         tma_load_3d(sK + s * C::TILE_BYTES + a * C::ATOM_BYTES, &tmK, &k_full[s], a * C::AW,
                                     p.kv_head0 + w.kvh, (w.j0 + j) * kTileN);
                     last_use[s] = u;
-                    if (j == 0 && w.hasB && !load_q(1)) { ok = false; break; }
+                    if (j == 0 && w.hasB && w.nB > 0 && !load_q(1)) { ok = false; break; }
                 }
                 if (!ok) break;
             }
@@ -380,10 +402,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int s = gk % C::KST, u = gk / C::KST;
             // A tile's last PV falls on the boundary when its key range ends the
             // union; B's always does (its range ends at its own diagonal tile).
-            const bool pvA = have_cur && cur.nA == nu;
-            const bool pvB = have_cur && cur.hasB;
-            const bool sA = have_nxt;
-            const bool sB = have_nxt && nxt.hasB && nxt.bstart == 0;
+            const bool pvA = have_cur && cur.nA > 0 && cur.nA == nu;
+            const bool pvB = have_cur && cur.hasB && cur.nB > 0;
+            const bool sA = have_nxt && nxt.nA > 0;
+            const bool sB = have_nxt && nxt.hasB && nxt.nB > 0 && nxt.bstart == 0;
             if (pvA || pvB) ok = mbar_wait_warp(&v_full[sp], up & 1, wc);
             if (ok && sA) ok = mbar_wait_warp(&k_full[s], u & 1, wc);
             if (ok && pvA) {
@@ -411,7 +433,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     umma_commit_elect(&o_done[1]);
                 }
             }
-            if (ok && have_nxt && nxt.hasB) {
+            if (ok && have_nxt && nxt.hasB && nxt.nB > 0) {
                 ok = mbar_wait_warp(&q_full[1], qcount[1] & 1, wc);
                 ++qcount[1];
             }
@@ -494,13 +516,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive(&item_empty[n & 1]);
             if (w.idx < 0) break;
             const int n_it = x == 0 ? w.nA : w.nB;
-            if (n_it == 0) continue;
-            const int first_union = x == 0 ? 0 : w.bstart;
             const int hx = x == 0 ? w.hA : w.hB;
             const int i = (x == 0 ? w.tA : w.tB) * kTileM + r;
-            const bool valid = i < p.N;
-            const int lo = valid ? p.doc_start[i] : i;
-            const int hi = i;
+            const bool valid = i >= p.q_lo && i < p.q_end && (x == 0 || w.hasB);
+            if (n_it == 0) {
+                // no key of the window for this tile: O = 0, LSE = -inf
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + static_cast<int64_t>(i - p.q_lo) * p.o_row_elems +
+                                                           static_cast<int64_t>(p.o_head0 + hx) * D);
+#pragma unroll
+                    for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+                    p.lse[static_cast<int64_t>(hx) * p.lse_ld + (i - p.q_lo)] = -CUDART_INF_F;
+                }
+                continue;
+            }
+            const int first_union = x == 0 ? 0 : w.bstart;
+            // keys this row may see: its document's, up to itself, inside the key window
+            const int lo = valid ? max(p.doc_start[i], p.kv_lo) : i;
+            const int hi = min(i, p.kv_hi - 1);
             float ms = -CUDART_INF_F;   // exponent offset in use (scaled log2 units)
             float l = 0.f;
             for (int it = 0; it < n_it; ++it) {
@@ -605,8 +638,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!ok || !mbar_wait_warp(&o_done[x], ocount & 1, wc)) { ok = false; break; }
             ++ocount;
             tc_fence_after();
-            const float inv_l = 1.f / l;
-            __nv_bfloat16 *orow = p.o + static_cast<int64_t>(i) * p.o_row_elems +
+            // A row that saw no key (possible only with a key window) never raised its
+            // running max above -inf: O = 0, LSE = -inf. (Its l need not be 0: the
+            // FMA-pipe exponential gives 2^-125 rather than 0 for masked columns.)
+            const bool seen = ms != -CUDART_INF_F;
+            const float inv_l = seen ? 1.f / l : 0.f;
+            __nv_bfloat16 *orow = p.o + static_cast<int64_t>(i - p.q_lo) * p.o_row_elems +
                                   static_cast<int64_t>(p.o_head0 + hx) * D;
             // the whole O row in one round trip (up to two x64 loads, one wait)
             uint32_t orw[D];
@@ -632,7 +669,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
                 }
             }
-            if (valid) p.lse[static_cast<int64_t>(hx) * p.N + i] = (ms + __log2f(l)) * 0.69314718055994530942f;
+            if (valid)
+                p.lse[static_cast<int64_t>(hx) * p.lse_ld + (i - p.q_lo)] =
+                    seen ? (ms + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
             tc_fence_before();
         }
     }
@@ -666,7 +705,15 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.o_head0 = a.o_head0;
     p.lse = a.lse;
     p.N = static_cast<int>(a.N);
-    p.T = static_cast<int>(ceil_div(a.N, kTileM));
+    p.q_tile0 = static_cast<int>(a.q_lo / kTileM);
+    p.T = static_cast<int>(ceil_div(a.q_hi, kTileM)) - p.q_tile0;
+    p.q_lo = static_cast<int>(a.q_lo);
+    p.q_end = static_cast<int>(a.q_hi);
+    p.lse_ld = static_cast<int>(a.lse_ld);
+    p.kv_lo = static_cast<int>(a.kv_lo);
+    p.kv_hi = static_cast<int>(a.kv_hi);
+    p.kvlo_t = static_cast<int>(a.kv_lo / kTileN);
+    p.kvhi_t = a.kv_hi > 0 ? static_cast<int>((a.kv_hi - 1) / kTileN) : -1;
     p.Hl = a.Hl;
     p.Hkvl = a.Hkvl;
     p.q_head0 = a.q_head0;
@@ -695,7 +742,20 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     // persistent: one CTA per SM (each needs a whole SM's tensor memory)
     const int sms = (dev < 64 && sm_count[dev] > 0) ? sm_count[dev] : 148;
     const int grid = p.items < sms ? p.items : sms;
-    attn_fwd_kernel<D><<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    // programmatic dependent launch: the prologue (barriers, tensor memory,
+    // descriptor prefetch) overlaps the doc-bounds kernel before it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kFwdThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D>, tq, tk, tv, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

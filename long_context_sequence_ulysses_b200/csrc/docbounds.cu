@@ -1,5 +1,5 @@
 // docbounds.cu -- per-token document starts and per-tile key ranges from
-// position_ids, plus the longest-first tile schedule.
+// position_ids, plus the longest-first tile schedule, in one launch.
 //
 // Packed documents are masked through position ids rather than a 4-D mask
 // (page "Ulysses verteilt Millionen-Token-Kontexte auf mehrere GPUs", section
@@ -10,18 +10,28 @@
 // [doc_start[i], i]; since doc_start never decreases, a 128-row query tile
 // starting at r0 needs key tiles doc_start[r0]/128 .. r0/128 and nothing else.
 //
-// Kernels: a block-local scan, a fix-up with the carry of earlier blocks
-// (which also writes each query tile's first key), for the backward the last
-// query row of each key tile (a binary search over doc_start), and a counting
-// sort of the scheduling units by work, heaviest first: query tiles (the
-// backward, and a forward whose items pair two heads of one KV group), pairs
-// of consecutive query tiles (a forward with an odd group size), and key
-// tiles (the backward).
+// One CTA of 1024 threads does all of it, so an attention call costs a single
+// small launch before its main kernel (which is launched as a programmatic
+// dependent of this one and runs its prologue meanwhile):
+//   1. the scan, 16384 tokens per pass: each warp scans 512 consecutive tokens
+//      (16 coalesced rows of 32), warp totals are scanned by warp 0, and the
+//      running maximum carries from pass to pass; every token costs O(1);
+//   2. for the backward, the last query row of each key tile (a binary search
+//      over doc_start);
+//   3. a counting sort of the scheduling units by work, heaviest first: query
+//      tiles (the backward, and a forward whose items pair two heads of one KV
+//      group), pairs of consecutive query tiles (a forward with an odd group
+//      size), and key tiles (the backward).
 #include "ulysses_internal.cuh"
 
 namespace uly {
 
 namespace {
+
+constexpr int kDbThreads = 1024;
+constexpr int kDbWarps = kDbThreads / 32;
+constexpr int kDbRows = 16;                              // rows of 32 tokens per warp and pass
+constexpr int kDbPass = kDbThreads * kDbRows;            // tokens per pass
 
 __device__ __forceinline__ int warp_incl_max(int v)
 {
@@ -33,96 +43,50 @@ __device__ __forceinline__ int warp_incl_max(int v)
     return v;
 }
 
-// Block-local inclusive max-scan over kScanBlock tokens (one per thread).
-__global__ void __launch_bounds__(kScanBlock) doc_scan_kernel(const int32_t *__restrict__ pos, int64_t N,
-                                                             int32_t *__restrict__ doc_start,
-                                                             int32_t *__restrict__ block_agg,
-                                                             uint32_t *__restrict__ status)
-{
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        status[0] = 0u;   // fresh status for this call
-        status[1] = 0u;   // work counter of the persistent forward kernel
-    }
-    __shared__ int warp_max[kScanBlock / 32];
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
-    int v = (i < N && pos[i] == 0) ? static_cast<int>(i) : 0;
-    v = warp_incl_max(v);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane == 31) warp_max[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_max[lane];
-        w = warp_incl_max(w);
-        warp_max[lane] = w;
-    }
-    __syncthreads();
-    if (warp > 0) v = max(v, warp_max[warp - 1]);
-    if (i < N) doc_start[i] = v;
-    if (threadIdx.x == kScanBlock - 1) block_agg[blockIdx.x] = v;
-}
-
-// Adds the carry of all earlier blocks and records each query tile's first key.
-__global__ void __launch_bounds__(kScanBlock) doc_fixup_kernel(int64_t N, int32_t *__restrict__ doc_start,
-                                                              const int32_t *__restrict__ block_agg,
-                                                              int32_t *__restrict__ tile_lo)
-{
-    __shared__ int red[kScanBlock / 32];
-    int c = 0;
-    for (int b = threadIdx.x; b < static_cast<int>(blockIdx.x); b += kScanBlock) c = max(c, block_agg[b]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c = max(c, __shfl_xor_sync(0xffffffffu, c, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        int w = red[threadIdx.x];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
-        if (threadIdx.x == 0) red[0] = w;
-    }
-    __syncthreads();
-    const int carry = red[0];
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
-    if (i < N) {
-        const int v = max(doc_start[i], carry);
-        doc_start[i] = v;
-        if ((i % kTileM) == 0) tile_lo[i / kTileM] = v;
-    }
-}
-
 // For key tile t: one past the last query row whose document reaches a key of
 // the tile, i.e. the number of rows i with doc_start[i] <= min(t*128+127, N-1).
-__global__ void kv_qend_kernel(int64_t N, int T, const int32_t *__restrict__ doc_start, int32_t *__restrict__ kv_qend)
+__device__ __forceinline__ int key_tile_qend(int64_t N, int t, const int32_t *doc_start)
 {
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
     const int64_t last_key = min(static_cast<int64_t>(t) * kTileN + kTileN - 1, N - 1);
     int64_t lo = last_key, hi = N;   // doc_start[last_key] <= last_key always holds
     while (hi - lo > 1) {            // invariant: doc_start[lo] <= last_key, doc_start[hi] > last_key (or hi == N)
         const int64_t mid = (lo + hi) >> 1;
         if (doc_start[mid] <= last_key) lo = mid; else hi = mid;
     }
-    kv_qend[t] = static_cast<int32_t>(hi);
+    return static_cast<int>(hi);
 }
 
-// Work of one scheduling unit. kQueryPairs: unit u is the pair of query
-// tiles (2u, 2u+1), work = key tiles visited by both (src = tile_lo, each
-// query tile's first key). kQueryTiles: unit t is query tile t, work = key
-// tiles it visits. kKeyTiles: unit t is key tile t, work = query tiles that
-// visit it (src = kv_qend).
+// Work of one scheduling unit, in key tiles inside the key window.
+// kQueryPairs: unit u is the pair of query tiles (q_tile0 + 2u, q_tile0 + 2u + 1),
+// work = key tiles visited by both (src = tile_lo, each query tile's first
+// key); the order lists u. kQueryTiles: unit u is query tile q_tile0 + u, work
+// = key tiles it visits; the order lists the tile itself. kKeyTiles: unit t is
+// key tile t, work = query tiles that visit it (src = kv_qend).
 enum class Unit { kQueryPairs, kQueryTiles, kKeyTiles };
 
-template <Unit kUnit>
-__device__ __forceinline__ int unit_work(int t, int T, const int32_t *__restrict__ src)
+__device__ __forceinline__ int query_tile_work(int t, const int32_t *tile_lo, const DbWindow &w)
 {
-    if (kUnit == Unit::kKeyTiles) return static_cast<int>((src[t] + kTileM - 1) / kTileM) - t;
-    if (kUnit == Unit::kQueryTiles) return t - src[t] / kTileN + 1;
-    const int ta = 2 * t, tb = 2 * t + 1;
-    int w = ta - src[ta] / kTileN + 1;
-    if (tb < T) w += tb - src[tb] / kTileN + 1;
-    return w;
+    return max(0, min(t, w.kvhi_t) - max(tile_lo[t] / kTileN, w.kvlo_t) + 1);
 }
 
-// Exclusive prefix sum over the 1024 threads of a block (warp shuffles, then
+template <Unit kUnit>
+__device__ __forceinline__ int unit_work(int u, const int32_t *src, const DbWindow &w)
+{
+    if (kUnit == Unit::kKeyTiles) return static_cast<int>((src[u] + kTileM - 1) / kTileM) - u;
+    if (kUnit == Unit::kQueryTiles) return query_tile_work(w.q_tile0 + u, src, w);
+    const int ta = w.q_tile0 + 2 * u, tb = ta + 1;
+    int work = query_tile_work(ta, src, w);
+    if (tb < w.q_tile0 + w.q_tiles) work += query_tile_work(tb, src, w);
+    return work;
+}
+
+template <Unit kUnit>
+__device__ __forceinline__ int unit_label(int u, const DbWindow &w)
+{
+    return kUnit == Unit::kQueryTiles ? w.q_tile0 + u : u;
+}
+
+// Exclusive prefix sum over the 1024 threads of the block (warp shuffles, then
 // the 32 warp totals in warp 0). warp_tot: 32 ints of shared memory.
 __device__ __forceinline__ int block_excl_sum_1024(int v, int *warp_tot)
 {
@@ -151,30 +115,27 @@ __device__ __forceinline__ int block_excl_sum_1024(int v, int *warp_tot)
 }
 
 // Largest work value whose histogram is kept in shared memory.
-constexpr int kOrderSmemWork = 11999;   // 48 KB of static shared memory with warp_tot
+constexpr int kOrderSmemWork = 11999;
 
 // Counting sort of `units` scheduling units by work (in [0, max_work]),
-// heaviest first. One CTA of 1024 threads; the histogram lives in shared
-// memory up to kOrderSmemWork, else in global scratch [max_work + 1]. Units
-// of equal work are placed in arrival order of the atomics (any order is a
-// valid schedule).
+// heaviest first, by the whole block. The histogram lives in shared memory up
+// to kOrderSmemWork, else in global scratch [max_work + 1]. Units of equal
+// work are placed in arrival order of the atomics (any order is a valid
+// schedule).
 template <Unit kUnit>
-__global__ void __launch_bounds__(1024) unit_order_kernel(int units, int T, int max_work,
-                                                         const int32_t *__restrict__ src,
-                                                         int32_t *__restrict__ ghist, int32_t *__restrict__ order)
+__device__ void unit_order(int units, const DbWindow &win, int max_work, const int32_t *src, int *shist,
+                           int32_t *ghist, int *warp_tot, int32_t *order)
 {
-    __shared__ int shist[kOrderSmemWork + 1];
-    __shared__ int warp_tot[32];
     int *hist = max_work <= kOrderSmemWork ? shist : ghist;
     const int tid = threadIdx.x;
-    for (int w = tid; w <= max_work; w += 1024) hist[w] = 0;
+    for (int w = tid; w <= max_work; w += kDbThreads) hist[w] = 0;
     __syncthreads();
-    for (int t = tid; t < units; t += 1024) atomicAdd(&hist[unit_work<kUnit>(t, T, src)], 1);
+    for (int t = tid; t < units; t += kDbThreads) atomicAdd(&hist[unit_work<kUnit>(t, src, win)], 1);
     __syncthreads();
     // Exclusive prefix over work values in DESCENDING order: the slot of the
     // first unit with work w is the number of units with work > w. Thread tid
     // owns a contiguous segment of work values counted from the top.
-    const int per = (max_work + 1 + 1023) / 1024;
+    const int per = (max_work + 1 + kDbThreads - 1) / kDbThreads;
     const int hi = max_work - tid * per;     // segment covers work values hi, hi-1, ..., hi-per+1
     int sum = 0;
     for (int k = 0; k < per; ++k) {
@@ -191,44 +152,109 @@ __global__ void __launch_bounds__(1024) unit_order_kernel(int units, int T, int 
         }
     }
     __syncthreads();
-    for (int t = tid; t < units; t += 1024) {
-        const int p = atomicAdd(&hist[unit_work<kUnit>(t, T, src)], 1);
-        order[p] = t;
+    for (int t = tid; t < units; t += kDbThreads) {
+        const int p = atomicAdd(&hist[unit_work<kUnit>(t, src, win)], 1);
+        order[p] = unit_label<kUnit>(t, win);
     }
+    __syncthreads();
+}
+
+struct DbArgs {
+    const int32_t *pos;
+    int64_t N;
+    int T;
+    int32_t *doc_start, *tile_lo, *q_order, *kv_qend, *kv_order, *ghist;
+    uint32_t *status;
+    int backward, fwd_tile_pairs;
+    DbWindow win;
+};
+
+__global__ void __launch_bounds__(kDbThreads, 1) docbounds_kernel(const DbArgs a)
+{
+    // The attention kernel that follows may start its prologue now; it reads
+    // nothing this kernel writes before its grid-dependency wait.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ int shist[kOrderSmemWork + 1];
+    __shared__ int wtot[kDbWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        a.status[0] = 0u;   // fresh status for this call
+        a.status[1] = 0u;   // work counter of the persistent forward kernel
+    }
+
+    // ---- 1. doc_start scan and each query tile's first key
+    int carry = 0;   // largest index of a 0 id in earlier passes (0 if none)
+    for (int64_t base = 0; base < a.N; base += kDbPass) {
+        const int64_t wbase = base + static_cast<int64_t>(warp) * (32 * kDbRows) + lane;
+        int v[kDbRows];
+#pragma unroll
+        for (int k = 0; k < kDbRows; ++k) {
+            const int64_t j = wbase + 32 * k;
+            v[k] = (j < a.N && a.pos[j] == 0) ? static_cast<int>(j) : 0;
+        }
+        int run = 0;   // maximum over this warp's earlier rows
+#pragma unroll
+        for (int k = 0; k < kDbRows; ++k) {
+            const int x = max(warp_incl_max(v[k]), run);
+            v[k] = x;
+            run = __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) wtot[warp] = run;
+        __syncthreads();
+        if (warp == 0) wtot[lane] = warp_incl_max(wtot[lane]);
+        __syncthreads();
+        const int pre = max(carry, warp > 0 ? wtot[warp - 1] : 0);
+#pragma unroll
+        for (int k = 0; k < kDbRows; ++k) {
+            const int64_t j = wbase + 32 * k;
+            if (j < a.N) {
+                const int ds = max(v[k], pre);
+                a.doc_start[j] = ds;
+                if ((j & (kTileM - 1)) == 0) a.tile_lo[j / kTileM] = ds;
+            }
+        }
+        carry = max(carry, wtot[kDbWarps - 1]);
+        __syncthreads();   // wtot is rewritten by the next pass
+    }
+    // (the block's global writes above are visible to all its threads after a barrier)
+    __syncthreads();
+
+    // ---- 2. backward: last query row of each key tile
+    if (a.backward) {
+        for (int t = threadIdx.x; t < a.T; t += kDbThreads) a.kv_qend[t] = key_tile_qend(a.N, t, a.doc_start);
+        __syncthreads();
+    }
+
+    // ---- 3. schedules, heaviest first
+    const int qt = a.win.q_tiles;
+    if (!a.backward && a.fwd_tile_pairs)
+        unit_order<Unit::kQueryPairs>((qt + 1) / 2, a.win, 2 * a.T, a.tile_lo, shist, a.ghist, wtot, a.q_order);
+    else
+        unit_order<Unit::kQueryTiles>(qt, a.win, a.T, a.tile_lo, shist, a.ghist, wtot, a.q_order);
+    if (a.backward)
+        unit_order<Unit::kKeyTiles>(a.T, a.win, a.T, a.kv_qend, shist, a.ghist, wtot, a.kv_order);
 }
 
 }  // namespace
 
 cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
-                             bool fwd_tile_pairs, cudaStream_t stream)
+                             bool fwd_tile_pairs, const DbWindow &win, cudaStream_t stream)
 {
-    const int64_t T = ceil_div(N, kTileM);
-    const int nb = static_cast<int>(ceil_div(N, kScanBlock));
-    int32_t *doc_start = reinterpret_cast<int32_t *>(ws + L.doc_start);
-    int32_t *tile_lo = reinterpret_cast<int32_t *>(ws + L.tile_lo);
-    int32_t *block_agg = reinterpret_cast<int32_t *>(ws + L.block_agg);
-    int32_t *scratch = reinterpret_cast<int32_t *>(ws + L.scratch);
-    doc_scan_kernel<<<nb, kScanBlock, 0, stream>>>(pos, N, doc_start, block_agg,
-                                                   reinterpret_cast<uint32_t *>(ws + L.status));
-    doc_fixup_kernel<<<nb, kScanBlock, 0, stream>>>(N, doc_start, block_agg, tile_lo);
-    if (!backward && fwd_tile_pairs) {
-        const int pairs = static_cast<int>(ceil_div(T, 2));
-        unit_order_kernel<Unit::kQueryPairs><<<1, 1024, 0, stream>>>(pairs, static_cast<int>(T),
-                                                                     static_cast<int>(2 * T), tile_lo, scratch,
-                                                                     reinterpret_cast<int32_t *>(ws + L.q_order));
-    } else {
-        unit_order_kernel<Unit::kQueryTiles><<<1, 1024, 0, stream>>>(static_cast<int>(T), static_cast<int>(T),
-                                                                     static_cast<int>(T), tile_lo, scratch,
-                                                                     reinterpret_cast<int32_t *>(ws + L.q_order));
-    }
-    if (backward) {
-        int32_t *kv_qend = reinterpret_cast<int32_t *>(ws + L.kv_qend);
-        kv_qend_kernel<<<static_cast<int>(ceil_div(T, 256)), 256, 0, stream>>>(N, static_cast<int>(T), doc_start,
-                                                                               kv_qend);
-        unit_order_kernel<Unit::kKeyTiles><<<1, 1024, 0, stream>>>(static_cast<int>(T), static_cast<int>(T),
-                                                                   static_cast<int>(T), kv_qend, scratch,
-                                                                   reinterpret_cast<int32_t *>(ws + L.kv_order));
-    }
+    DbArgs a;
+    a.pos = pos;
+    a.N = N;
+    a.T = static_cast<int>(ceil_div(N, kTileM));
+    a.doc_start = reinterpret_cast<int32_t *>(ws + L.doc_start);
+    a.tile_lo = reinterpret_cast<int32_t *>(ws + L.tile_lo);
+    a.q_order = reinterpret_cast<int32_t *>(ws + L.q_order);
+    a.kv_qend = backward ? reinterpret_cast<int32_t *>(ws + L.kv_qend) : nullptr;
+    a.kv_order = backward ? reinterpret_cast<int32_t *>(ws + L.kv_order) : nullptr;
+    a.ghist = reinterpret_cast<int32_t *>(ws + L.scratch);
+    a.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    a.backward = backward ? 1 : 0;
+    a.fwd_tile_pairs = fwd_tile_pairs ? 1 : 0;
+    a.win = win;
+    docbounds_kernel<<<1, kDbThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

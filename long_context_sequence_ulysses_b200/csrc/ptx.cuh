@@ -106,6 +106,12 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, W
     return ok;
 }
 
+// ---------------------------------------------------------------- grid dependencies
+// A kernel launched as a programmatic dependent of the previous one on its
+// stream may start while that one still runs; this waits until it has
+// completed and its memory writes are visible (a no-op without a dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m)
 {
@@ -125,6 +131,17 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// 4-D tiled load (same rules as tma_load_3d).
+__device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m, uint64_t *bar,
+                                            int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)),
+          "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
 
 // ---------------------------------------------------------------- tcgen05
 // Tensor memory allocation: executed by one full warp. The allocated column

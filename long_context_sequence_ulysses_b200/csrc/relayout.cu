@@ -7,6 +7,10 @@
 // whole sequence for heads [r*Hx/P, (r+1)*Hx/P). Head-to-sequence (step
 // 全体间通信复原) is the inverse.
 //
+// The exchanged heads may be a slice [head0, head0 + Hx) of wider
+// sequence-side rows of row_heads heads (one chunk of heads at a time, as the
+// head-chunked variant exchanges them), read or written in place.
+//
 // For a fixed destination rank r and token n the data moved is one contiguous
 // chunk of C = Hx/P*d*2 bytes on both sides, so each CTA streams the chunks of
 // consecutive tokens: the chunk-side run is contiguous, the sequence-side
@@ -47,10 +51,12 @@ struct RelayoutArgs {
     const uint4 *src;
     uint4 *dst;
     int64_t N;          // tokens
-    int64_t row_vecs;   // Hx*d/8: vectors per token row on the sequence side
+    int64_t row_vecs;   // vectors between consecutive token rows on the sequence side
+                        // (Hx*d/8, or more when the exchanged heads are a slice of wider rows)
     int C;              // Hx/P*d/8: vectors per chunk
     int rank0;
     int64_t head_rank_stride;
+    int64_t col0;       // first vector of the exchanged heads within a sequence-side row
     int tokens_per_iter;  // tokens covered by one CTA pass (kRelayoutThreads / C, >= 1)
     int e_iters;          // chunks wider than the CTA: ceil(C / kRelayoutThreads)
 };
@@ -70,7 +76,7 @@ __global__ void __launch_bounds__(kRelayoutThreads) relayout_kernel(RelayoutArgs
         e0 = t;
     }
     const int64_t head_base = (blockIdx.y) * a.head_rank_stride;
-    const int64_t seq_col = static_cast<int64_t>(r) * a.C;
+    const int64_t seq_col = a.col0 + static_cast<int64_t>(r) * a.C;
     const int64_t step = static_cast<int64_t>(gridDim.x) * a.tokens_per_iter;
 
     for (int ei = 0; ei < a.e_iters; ++ei) {
@@ -104,13 +110,14 @@ __global__ void __launch_bounds__(kRelayoutThreads) relayout_kernel(RelayoutArgs
 }  // namespace
 
 cudaError_t launch_relayout(bool to_head, const void *src, void *dst, int64_t N, int P, int Hx, int d, int rank,
-                            cudaStream_t stream, int num_sms)
+                            int row_heads, int head0, cudaStream_t stream, int num_sms)
 {
     RelayoutArgs a;
     a.src = static_cast<const uint4 *>(src);
     a.dst = static_cast<uint4 *>(dst);
     a.N = N;
-    a.row_vecs = static_cast<int64_t>(Hx) * d / 8;
+    a.row_vecs = static_cast<int64_t>(row_heads) * d / 8;
+    a.col0 = static_cast<int64_t>(head0) * d / 8;
     a.C = (Hx / P) * d / 8;
     const int nranks = rank < 0 ? P : 1;
     a.rank0 = rank < 0 ? 0 : rank;

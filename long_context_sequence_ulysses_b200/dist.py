@@ -160,12 +160,15 @@ def attention_forward_chunked(q_local: torch.Tensor, k_local: torch.Tensor, v_lo
     pos = gather_position_ids(pos_local, group)
 
     def start(c: int):
-        """Pack chunk c's Q, K, V and start their all-to-alls (asynchronous)."""
+        """Pack chunk c's Q, K, V and start their all-to-alls (asynchronous).
+        The CUDA pack reads the chunk's heads in place from the full shard."""
         inflight = []
         for x, h in ((q_local, Hc), (k_local, Hkvc), (v_local, Hkvc)):
-            xc = x[:, c * h:(c + 1) * h].contiguous()
-            send = _cuda_pack(xc, G) if pack is None else pack(xc, G)   # [G][N/G][h/G][d]
-            send = send.contiguous()
+            if pack is None:
+                import long_context_sequence_ulysses_b200 as U
+                send = U.seq_to_head(x, G, heads=(c * h, h))                # [G][N/G][h/G][d]
+            else:
+                send = pack(x[:, c * h:(c + 1) * h].contiguous(), G).contiguous()
             recv = torch.empty_like(send)
             work = dist.all_to_all_single(recv.view(torch.uint8), send.view(torch.uint8), group=group,
                                           async_op=True)
@@ -182,7 +185,15 @@ def attention_forward_chunked(q_local: torch.Tensor, k_local: torch.Tensor, v_lo
             work.wait()
         q, k, v = (recv.view(G * n_loc, recv.shape[2], d) for _, recv, _ in current)
         o, lse = attn(q, k, v, pos, scale=scale)
-        o_local[:, c * Hc:(c + 1) * Hc] = head_to_seq(o, group, unpack)
+        if unpack is None:
+            # second exchange, then the unpack writes this chunk's heads of o_local in place
+            send = o.contiguous().view(G, n_loc, o.shape[1], d)
+            recv = torch.empty_like(send)
+            dist.all_to_all_single(recv.view(torch.uint8), send.view(torch.uint8), group=group)
+            import long_context_sequence_ulysses_b200 as U
+            U.head_to_seq(recv, G, out=o_local, head0=c * Hc)
+        else:
+            o_local[:, c * Hc:(c + 1) * Hc] = head_to_seq(o, group, unpack)
         lses.append(lse)
         heads.append([c * Hc + rank * (Hc // G) + j for j in range(Hc // G)])
     return o_local, torch.stack(lses), pos, heads

@@ -31,7 +31,7 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     tolerance: per comparison, max |ref|, and the elements whose error is above
     the flat 2e-2 (allowed only where |ref| >= 4, by 2^-8 |ref|)."""
     try:
-        from helpers import GRAD_STATS, GRAD_FLAT_BELOW, MAX_ABS
+        from helpers import GRAD_BINS, GRAD_STATS, GRAD_FLAT_BELOW, MAX_ABS
     except Exception:  # pragma: no cover
         return
     if not GRAD_STATS:
@@ -42,5 +42,11 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     over = sum(s[3] for s in GRAD_STATS)
     tr.write_line(f"{len(GRAD_STATS)} comparisons, {tot} elements, {over} with |err| > {MAX_ABS} "
                   f"(flat bound asserted wherever |ref| < {GRAD_FLAT_BELOW})")
-    for name, mref, n, nover, ws in GRAD_STATS:
-        tr.write_line(f"  {name}: max|ref| {mref:.3g}, {nover}/{n} above flat, worst |err| at |ref|<4 {ws:.3e}")
+    edges = ", ".join(f"[{a:g},{b:g})" for a, b in zip(GRAD_BINS[:-1], GRAD_BINS[1:]))
+    worst = [max((s[5][i] for s in GRAD_STATS if s[5][i] is not None), default=None)
+             for i in range(len(GRAD_BINS) - 1)]
+    tr.write_line("worst |err| per |ref| bin " + edges + ": "
+                  + ", ".join("-" if w is None else f"{w:.3e}" for w in worst))
+    for name, mref, n, nover, ws, bins in GRAD_STATS:
+        tr.write_line(f"  {name}: max|ref| {mref:.3g}, {nover}/{n} above flat; worst |err| per bin "
+                      + ", ".join("-" if b is None else f"{b:.2e}" for b in bins))

@@ -236,3 +236,30 @@ def test_binding_checks_shapes_before_device():
         U.attn_bwd(**_bwd_ok())
     with pytest.raises(TypeError):
         U.attn_fwd_fused(**_fused_ok())
+
+
+def test_window_and_merge_argument_errors():
+    lib = _lib()
+    ws_ok = lib.ulysses_attn_workspace_bytes(256, 4, 2, 128, 0)
+
+    def rejects(f, args, code, text):
+        assert f(*args) == code
+        assert text in lib.ulysses_last_error(), lib.ulysses_last_error()
+
+    f = lib.ulysses_attn_fwd_window
+    wa = lambda ql, qh, kl, kh: (FAKE, FAKE, FAKE, FAKE, 256, 4, 2, 128, ql, qh, kl, kh, ctypes.c_float(0.0), FAKE,
+                                 FAKE, FAKE, ws_ok, None)
+    rejects(f, wa(-1, 10, 0, 256), -1, b"query window [-1, 10)")
+    rejects(f, wa(10, 5, 0, 256), -1, b"query window [10, 5)")
+    rejects(f, wa(0, 257, 0, 256), -1, b"query window [0, 257)")
+    rejects(f, wa(0, 256, 100, 50), -1, b"key window [100, 50)")
+    rejects(f, wa(0, 256, 0, 300), -1, b"key window [0, 300)")
+    assert f(*wa(64, 64, 0, 256)) == 0                            # empty query window: nothing to do
+    m = lib.ulysses_attn_merge
+    ma = lambda R, M, Hl, d, ld: (FAKE, FAKE, R, M, Hl, d, FAKE, FAKE, ld, None)
+    rejects(m, ma(0, 16, 4, 128, 16), -1, b"R=0 outside [1, 64]")
+    rejects(m, ma(65, 16, 4, 128, 16), -1, b"R=65")
+    rejects(m, ma(2, 16, 4, 96, 16), -1, b"d=96")
+    rejects(m, ma(2, 16, 4, 128, 15), -1, b"lse_ld=15 < M=16")
+    rejects(m, (FAKE_MIS, FAKE, 2, 16, 4, 128, FAKE, FAKE, 16, None), -1, b"16-byte aligned")
+    assert m(*ma(2, 0, 4, 128, 0)) == 0                           # no rows

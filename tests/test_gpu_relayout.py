@@ -94,3 +94,21 @@ def test_million_relayout_properties():
         assert np.array_equal(got.reshape(w.P, w.P * len(m), Hx // w.P, w.d).cpu().numpy().view(np.uint16), ref)
         del x, y, back
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("N,P,row_heads,head0,Hx,d", [(256, 2, 8, 4, 4, 32), (384, 4, 32, 8, 8, 128),
+                                                     (96, 1, 3, 1, 2, 64), (512, 8, 24, 16, 8, 128)])
+def test_head_slice_exchanges(N, P, row_heads, head0, Hx, d):
+    """The exchange of a slice of heads [head0, head0+Hx) of wider rows, read
+    and written in place: equal to the oracle's exchange of that slice, and
+    the unpack leaves the other heads of the destination untouched."""
+    import long_context_sequence_ulysses_b200 as U
+    x = normal_bf16((N, row_heads, d), seed=N + head0, device="cuda", stream_id=10)
+    y = U.seq_to_head(x, P, heads=(head0, Hx))
+    ref = oracle.seq_to_head(x[:, head0:head0 + Hx].contiguous(), N, P, Hx, d)
+    assert np.array_equal(_u16(y), ref)
+    out = torch.full_like(x, float("nan"))
+    U.head_to_seq(y, P, out=out, head0=head0)
+    assert np.array_equal(_u16(out[:, head0:head0 + Hx]), _u16(x[:, head0:head0 + Hx]))
+    rest = torch.cat([out[:, :head0], out[:, head0 + Hx:]], dim=1)
+    assert torch.isnan(rest.float()).all()

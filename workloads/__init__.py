@@ -14,6 +14,9 @@ Workloads (named by what they are):
 * ``million``   N=1048576, P=8, H=32 / Hkv=8, d=128, one document.
 * ``train``     N=65536, P=4, H=32 / Hkv=8, d=128, packed documents with
                 geometric lengths (mean 4096), forward + backward.
+* ``hybrid_kv2`` the llama8b shape with only 2 KV heads over P=8 ranks: fewer
+                KV heads than ranks, so Ulysses alone cannot split it; run as
+                the Ulysses x ring hybrid (2-way Ulysses, 4-way ring).
 
 Sequence sharding follows the page "Hugging Face并行加速：10倍提升超长序列训练效率",
 section "Ulysses的工作原理", step 序列分片: GPU i owns tokens [i*n/P, (i+1)*n/P).
@@ -42,6 +45,7 @@ class Workload:
     seed: int
     prescale: bool = False   # multiply Q/K/V by 1/sqrt(d) before the bf16 cast
     backward: bool = False   # the workload includes the backward pass
+    ulysses: int = 0         # > 0: Ulysses x ring hybrid with this Ulysses degree (ring degree P / ulysses)
 
     @property
     def Hl(self) -> int:
@@ -58,6 +62,7 @@ WORKLOADS: Dict[str, Workload] = {
     "long131k": Workload("long131k", 131072, 4, 32, 8, 128, "single", 2),
     "million": Workload("million", 1048576, 8, 32, 8, 128, "single", 3),
     "train": Workload("train", 65536, 4, 32, 8, 128, "geometric", 4, backward=True),
+    "hybrid_kv2": Workload("hybrid_kv2", 32768, 8, 32, 2, 128, "uniform", 5, prescale=True, ulysses=2),
 }
 
 
@@ -161,3 +166,20 @@ def random_case(N: int, H: int, Hkv: int, d: int, lengths: List[int], seed: int,
     if with_grad_out:
         out["do"] = normal_bf16((N, H, d), seed, device, None, STREAM_DO)
     return out
+
+
+STREAM_WQKV, STREAM_WO, STREAM_X = 5, 6, 7
+
+
+def projection_inputs(w: Workload, device="cpu", N: Optional[int] = None) -> dict:
+    """Synthetic layer inputs around the path: activations x [N][hidden] ~
+    N(0, 1) and random-init weights w_qkv [(H+2Hkv)d][hidden], w_o [hidden][Hd]
+    ~ N(0, 1/hidden) (hidden = H*d, as in the Llama-8B shape), all bf16."""
+    n = w.N if N is None else N
+    hidden = w.H * w.d
+    sc = 1.0 / math.sqrt(hidden)
+    return {
+        "x": normal_bf16((n, hidden), w.seed, device, None, STREAM_X),
+        "w_qkv": normal_bf16(((w.H + 2 * w.Hkv) * w.d, hidden), w.seed, device, sc, STREAM_WQKV),
+        "w_o": normal_bf16((hidden, w.H * w.d), w.seed, device, sc, STREAM_WO),
+    }
