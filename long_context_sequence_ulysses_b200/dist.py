@@ -183,7 +183,10 @@ def attention_forward_chunked(q_local: torch.Tensor, k_local: torch.Tensor, v_lo
         pending = start(c + 1) if c + 1 < chunks else None
         for work, _, _ in current:
             work.wait()
-        q, k, v = (recv.view(G * n_loc, recv.shape[2], d) for _, recv, _ in current)
+        # the send buffers are free once their exchange is done; keep only the received slices
+        recvs = [recv for _, recv, _ in current]
+        del current
+        q, k, v = (recv.view(G * n_loc, recv.shape[2], d) for recv in recvs)
         o, lse = attn(q, k, v, pos, scale=scale)
         if unpack is None:
             # second exchange, then the unpack writes this chunk's heads of o_local in place
@@ -196,4 +199,5 @@ def attention_forward_chunked(q_local: torch.Tensor, k_local: torch.Tensor, v_lo
             o_local[:, c * Hc:(c + 1) * Hc] = head_to_seq(o, group, unpack)
         lses.append(lse)
         heads.append([c * Hc + rank * (Hc // G) + j for j in range(Hc // G)])
+        del recvs, q, k, v, o
     return o_local, torch.stack(lses), pos, heads

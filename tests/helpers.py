@@ -15,14 +15,14 @@ MEAN_ABS = 2e-3
 # per-element bound is therefore 2e-2 + 2^-8 * |ref| (two such roundings), with
 # the same mean-abs 2e-3.
 GRAD_REL = 2.0 ** -8
-# Below this magnitude the flat bound alone must hold for gradients too: there
-# bf16 storage moves a value by at most 2^-9 * 2 = 0.004, and the relative
-# term (2^-8 |ref| < 0.008) is not needed. Between 2 and 4 a stored bf16 value
-# is already off by up to 0.008, and the bf16 P and dS operands of the
-# gradient products add about 2^-9 of the sum of |terms|, which with a GQA
-# group of 4-8 heads and long documents exceeds 2e-2 for a few elements (the
-# per-magnitude maxima are printed by conftest.py).
-GRAD_FLAT_BELOW = 2.0
+# Below this magnitude the flat bound alone must hold for gradients too. The
+# backward's own bf16 roundings (D from the bf16 O, P and dS as bf16 operands
+# of the tensor-core products) give errors that follow the size of the summed
+# terms rather than |ref|: an fp64 model with just those roundings already
+# reaches 1.9e-2 in dK at |ref| 1.6 and 1.1e-2 in dQ at |ref| 0.06
+# (tests/test_tolerance_model.py), so the flat 2e-2 is asserted only where
+# |ref| < 0.5, and the relative term carries the rest.
+GRAD_FLAT_BELOW = 0.5
 # |ref| bins of the per-magnitude error maxima
 GRAD_BINS = (0.0, 0.5, 1.0, 2.0, 4.0, float("inf"))
 # (name, max |ref|, elements, elements with |err| > MAX_ABS, worst |err| where
