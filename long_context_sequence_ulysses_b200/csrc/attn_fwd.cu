@@ -275,6 +275,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
             int kcount = 0;                  // K tiles loaded so far (ring position)
             int qcount[2] = {0, 0};          // Q_x tiles loaded so far
             int last_use[C::KST];
@@ -292,6 +293,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int f = 0; f < kItemInts; ++f) item_ring[slot * kItemInts + f] = wi[f];
                 mbar_arrive(&item_full[slot]);   // release: the fields are visible to every waiter
                 if (w.idx < 0) break;
+                // The item is known about two key steps before the current one ends,
+                // but its Q tiles and first K/V tiles can only be loaded into shared
+                // memory as the current item frees them: bring them into L2 now,
+                // so that those loads do not wait for HBM at the item boundary.
+#pragma unroll
+                for (int a = 0; a < C::NA; ++a) {
+                    if (w.nA > 0) tma_prefetch_3d(&tmQ, a * C::AW, p.q_head0 + w.hA, w.tA * kTileM);
+                    if (w.hasB && w.nB > 0) tma_prefetch_3d(&tmQ, a * C::AW, p.q_head0 + w.hB, w.tB * kTileM);
+                    for (int j = 0; j < 2 && j < w.n_union; ++j) {
+                        tma_prefetch_3d(&tmK, a * C::AW, p.kv_head0 + w.kvh, (w.j0 + j) * kTileN);
+                        tma_prefetch_3d(&tmV, a * C::AW, p.kv_head0 + w.kvh, (w.j0 + j) * kTileN);
+                    }
+                }
                 // Q_A, K_0, Q_B, K_1, K_2, ...: the next item's first S (tile A) needs
                 // only Q_A and K_0, and Q_B's buffer is freed last (by B's final S).
                 auto load_q = [&](int x) -> bool {

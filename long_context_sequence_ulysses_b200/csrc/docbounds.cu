@@ -1,5 +1,5 @@
 // docbounds.cu -- per-token document starts and per-tile key ranges from
-// position_ids, plus the longest-first tile schedule, in one launch.
+// position_ids, plus the longest-first tile schedule.
 //
 // Packed documents are masked through position ids rather than a 4-D mask
 // (page "Ulysses verteilt Millionen-Token-Kontexte auf mehrere GPUs", section
@@ -10,18 +10,21 @@
 // [doc_start[i], i]; since doc_start never decreases, a 128-row query tile
 // starting at r0 needs key tiles doc_start[r0]/128 .. r0/128 and nothing else.
 //
-// One CTA of 1024 threads does all of it, so an attention call costs a single
-// small launch before its main kernel (which is launched as a programmatic
-// dependent of this one and runs its prologue meanwhile):
-//   1. the scan, 16384 tokens per pass: each warp scans 512 consecutive tokens
-//      (16 coalesced rows of 32), warp totals are scanned by warp 0, and the
-//      running maximum carries from pass to pass; every token costs O(1);
-//   2. for the backward, the last query row of each key tile (a binary search
-//      over doc_start);
-//   3. a counting sort of the scheduling units by work, heaviest first: query
-//      tiles (the backward, and a forward whose items pair two heads of one KV
-//      group), pairs of consecutive query tiles (a forward with an odd group
-//      size), and key tiles (the backward).
+// Kernels (all short; measured faster than one CTA doing everything, whose
+// serial passes over the ids sit on the attention's critical path):
+//   1. doc_scan: block-local scan of 1024 tokens per block, block maxima;
+//   2. (more than 1024 blocks only) carry_prefix: one CTA turns the block maxima
+//      into each block's carry, so that the total work stays O(N);
+//   3. doc_fixup: adds the carry of earlier blocks, writes each query tile's
+//      first key;
+//   4. backward only: the last query row of each key tile (binary search);
+//   5. unit_order: a counting sort of the scheduling units by work, heaviest
+//      first -- query tiles (the backward, and a forward whose items pair two
+//      heads of one KV group), pairs of consecutive query tiles (a forward with
+//      an odd group size), key tiles (the backward) -- counting only key tiles
+//      inside the forward's key window. The forward's attention kernel is
+//      launched as a programmatic dependent of the last sort, which lets it
+//      start its prologue while the sort runs.
 #include "ulysses_internal.cuh"
 
 namespace uly {
@@ -29,9 +32,6 @@ namespace uly {
 namespace {
 
 constexpr int kDbThreads = 1024;
-constexpr int kDbWarps = kDbThreads / 32;
-constexpr int kDbRows = 16;                              // rows of 32 tokens per warp and pass
-constexpr int kDbPass = kDbThreads * kDbRows;            // tokens per pass
 
 __device__ __forceinline__ int warp_incl_max(int v)
 {
@@ -41,6 +41,91 @@ __device__ __forceinline__ int warp_incl_max(int v)
         if ((threadIdx.x & 31) >= o) v = max(v, u);
     }
     return v;
+}
+
+// Inclusive max-scan of v over the 1024 threads of the block. wmax: 32 ints of shared memory.
+__device__ __forceinline__ int block_incl_max_1024(int v, int *wmax)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_incl_max(v);
+    if (lane == 31) wmax[warp] = v;
+    __syncthreads();
+    if (warp == 0) wmax[lane] = warp_incl_max(wmax[lane]);
+    __syncthreads();
+    if (warp > 0) v = max(v, wmax[warp - 1]);
+    __syncthreads();   // wmax may be reused after this
+    return v;
+}
+
+// 1. Block-local inclusive max-scan over kScanBlock tokens (one per thread).
+__global__ void __launch_bounds__(kScanBlock) doc_scan_kernel(const int32_t *__restrict__ pos, int64_t N,
+                                                             int32_t *__restrict__ doc_start,
+                                                             int32_t *__restrict__ block_agg,
+                                                             uint32_t *__restrict__ status)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        status[0] = 0u;   // fresh status for this call
+        status[1] = 0u;   // work counter of the persistent forward kernel
+    }
+    __shared__ int wmax[32];
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
+    const int v = block_incl_max_1024((i < N && pos[i] == 0) ? static_cast<int>(i) : 0, wmax);
+    if (i < N) doc_start[i] = v;
+    if (threadIdx.x == kScanBlock - 1) block_agg[blockIdx.x] = v;
+}
+
+// 2. More than kScanBlock blocks: block b's carry = max of block_agg[0..b), by
+// one CTA walking the maxima 1024 at a time (O(nb) in all).
+__global__ void __launch_bounds__(kScanBlock) carry_prefix_kernel(const int32_t *__restrict__ block_agg, int nb,
+                                                                 int32_t *__restrict__ block_carry)
+{
+    __shared__ int wmax[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int run = 0;   // maximum of the blocks of earlier passes
+    for (int base = 0; base < nb; base += kScanBlock) {
+        const int b = base + threadIdx.x;
+        const int incl = block_incl_max_1024(b < nb ? block_agg[b] : 0, wmax);   // wmax: prefix over warps
+        const int prev = __shfl_up_sync(0xffffffffu, incl, 1);
+        const int excl = lane ? prev : (warp ? wmax[warp - 1] : 0);
+        if (b < nb) block_carry[b] = max(run, excl);
+        run = max(run, wmax[31]);
+        __syncthreads();   // wmax is rewritten by the next pass
+    }
+}
+
+// 3. Adds the carry of all earlier blocks and records each query tile's first
+// key. With at most kScanBlock blocks every block reduces the maxima before it
+// (one load per thread); beyond that it reads the carry computed in step 2.
+__global__ void __launch_bounds__(kScanBlock) doc_fixup_kernel(int64_t N, int nb, int32_t *__restrict__ doc_start,
+                                                              const int32_t *__restrict__ block_agg,
+                                                              const int32_t *__restrict__ block_carry,
+                                                              int32_t *__restrict__ tile_lo)
+{
+    __shared__ int red[32];
+    int carry;
+    if (nb <= kScanBlock) {
+        int c = threadIdx.x < static_cast<int>(blockIdx.x) ? block_agg[threadIdx.x] : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c = max(c, __shfl_xor_sync(0xffffffffu, c, o));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            int w = red[threadIdx.x];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
+            if (threadIdx.x == 0) red[0] = w;
+        }
+        __syncthreads();
+        carry = red[0];
+    } else {
+        carry = block_carry[blockIdx.x];
+    }
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanBlock + threadIdx.x;
+    if (i < N) {
+        const int v = max(doc_start[i], carry);
+        doc_start[i] = v;
+        if ((i % kTileM) == 0) tile_lo[i / kTileM] = v;
+    }
 }
 
 // For key tile t: one past the last query row whose document reaches a key of
@@ -159,80 +244,26 @@ __device__ void unit_order(int units, const DbWindow &win, int max_work, const i
     __syncthreads();
 }
 
-struct DbArgs {
-    const int32_t *pos;
-    int64_t N;
-    int T;
-    int32_t *doc_start, *tile_lo, *q_order, *kv_qend, *kv_order, *ghist;
-    uint32_t *status;
-    int backward, fwd_tile_pairs;
-    DbWindow win;
-};
-
-__global__ void __launch_bounds__(kDbThreads, 1) docbounds_kernel(const DbArgs a)
+// 4. For each key tile: one past the last query row that reaches it.
+__global__ void kv_qend_kernel(int64_t N, int T, const int32_t *__restrict__ doc_start, int32_t *__restrict__ kv_qend)
 {
-    // The attention kernel that follows may start its prologue now; it reads
-    // nothing this kernel writes before its grid-dependency wait.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t < T) kv_qend[t] = key_tile_qend(N, t, doc_start);
+}
+
+// 5. One schedule. `trigger`: the kernel after this one (the forward's
+// attention kernel) may start its prologue right away; it reads this kernel's
+// results only after its grid-dependency wait.
+template <Unit kUnit>
+__global__ void __launch_bounds__(kDbThreads, 1) unit_order_kernel(int units, DbWindow win, int max_work,
+                                                                  const int32_t *__restrict__ src,
+                                                                  int32_t *__restrict__ ghist,
+                                                                  int32_t *__restrict__ order, int trigger)
+{
+    if (trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ int shist[kOrderSmemWork + 1];
-    __shared__ int wtot[kDbWarps];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) {
-        a.status[0] = 0u;   // fresh status for this call
-        a.status[1] = 0u;   // work counter of the persistent forward kernel
-    }
-
-    // ---- 1. doc_start scan and each query tile's first key
-    int carry = 0;   // largest index of a 0 id in earlier passes (0 if none)
-    for (int64_t base = 0; base < a.N; base += kDbPass) {
-        const int64_t wbase = base + static_cast<int64_t>(warp) * (32 * kDbRows) + lane;
-        int v[kDbRows];
-#pragma unroll
-        for (int k = 0; k < kDbRows; ++k) {
-            const int64_t j = wbase + 32 * k;
-            v[k] = (j < a.N && a.pos[j] == 0) ? static_cast<int>(j) : 0;
-        }
-        int run = 0;   // maximum over this warp's earlier rows
-#pragma unroll
-        for (int k = 0; k < kDbRows; ++k) {
-            const int x = max(warp_incl_max(v[k]), run);
-            v[k] = x;
-            run = __shfl_sync(0xffffffffu, x, 31);
-        }
-        if (lane == 0) wtot[warp] = run;
-        __syncthreads();
-        if (warp == 0) wtot[lane] = warp_incl_max(wtot[lane]);
-        __syncthreads();
-        const int pre = max(carry, warp > 0 ? wtot[warp - 1] : 0);
-#pragma unroll
-        for (int k = 0; k < kDbRows; ++k) {
-            const int64_t j = wbase + 32 * k;
-            if (j < a.N) {
-                const int ds = max(v[k], pre);
-                a.doc_start[j] = ds;
-                if ((j & (kTileM - 1)) == 0) a.tile_lo[j / kTileM] = ds;
-            }
-        }
-        carry = max(carry, wtot[kDbWarps - 1]);
-        __syncthreads();   // wtot is rewritten by the next pass
-    }
-    // (the block's global writes above are visible to all its threads after a barrier)
-    __syncthreads();
-
-    // ---- 2. backward: last query row of each key tile
-    if (a.backward) {
-        for (int t = threadIdx.x; t < a.T; t += kDbThreads) a.kv_qend[t] = key_tile_qend(a.N, t, a.doc_start);
-        __syncthreads();
-    }
-
-    // ---- 3. schedules, heaviest first
-    const int qt = a.win.q_tiles;
-    if (!a.backward && a.fwd_tile_pairs)
-        unit_order<Unit::kQueryPairs>((qt + 1) / 2, a.win, 2 * a.T, a.tile_lo, shist, a.ghist, wtot, a.q_order);
-    else
-        unit_order<Unit::kQueryTiles>(qt, a.win, a.T, a.tile_lo, shist, a.ghist, wtot, a.q_order);
-    if (a.backward)
-        unit_order<Unit::kKeyTiles>(a.T, a.win, a.T, a.kv_qend, shist, a.ghist, wtot, a.kv_order);
+    __shared__ int wtot[32];
+    unit_order<kUnit>(units, win, max_work, src, shist, ghist, wtot, order);
 }
 
 }  // namespace
@@ -240,21 +271,32 @@ __global__ void __launch_bounds__(kDbThreads, 1) docbounds_kernel(const DbArgs a
 cudaError_t launch_docbounds(const int32_t *pos, int64_t N, char *ws, const WsLayout &L, bool backward,
                              bool fwd_tile_pairs, const DbWindow &win, cudaStream_t stream)
 {
-    DbArgs a;
-    a.pos = pos;
-    a.N = N;
-    a.T = static_cast<int>(ceil_div(N, kTileM));
-    a.doc_start = reinterpret_cast<int32_t *>(ws + L.doc_start);
-    a.tile_lo = reinterpret_cast<int32_t *>(ws + L.tile_lo);
-    a.q_order = reinterpret_cast<int32_t *>(ws + L.q_order);
-    a.kv_qend = backward ? reinterpret_cast<int32_t *>(ws + L.kv_qend) : nullptr;
-    a.kv_order = backward ? reinterpret_cast<int32_t *>(ws + L.kv_order) : nullptr;
-    a.ghist = reinterpret_cast<int32_t *>(ws + L.scratch);
-    a.status = reinterpret_cast<uint32_t *>(ws + L.status);
-    a.backward = backward ? 1 : 0;
-    a.fwd_tile_pairs = fwd_tile_pairs ? 1 : 0;
-    a.win = win;
-    docbounds_kernel<<<1, kDbThreads, 0, stream>>>(a);
+    const int T = static_cast<int>(ceil_div(N, kTileM));
+    const int nb = static_cast<int>(ceil_div(N, kScanBlock));
+    int32_t *doc_start = reinterpret_cast<int32_t *>(ws + L.doc_start);
+    int32_t *tile_lo = reinterpret_cast<int32_t *>(ws + L.tile_lo);
+    int32_t *q_order = reinterpret_cast<int32_t *>(ws + L.q_order);
+    int32_t *block_agg = reinterpret_cast<int32_t *>(ws + L.block_agg);
+    int32_t *block_carry = reinterpret_cast<int32_t *>(ws + L.block_carry);
+    int32_t *ghist = reinterpret_cast<int32_t *>(ws + L.scratch);
+    doc_scan_kernel<<<nb, kScanBlock, 0, stream>>>(pos, N, doc_start, block_agg,
+                                                   reinterpret_cast<uint32_t *>(ws + L.status));
+    if (nb > kScanBlock) carry_prefix_kernel<<<1, kScanBlock, 0, stream>>>(block_agg, nb, block_carry);
+    doc_fixup_kernel<<<nb, kScanBlock, 0, stream>>>(N, nb, doc_start, block_agg, block_carry, tile_lo);
+    if (backward) {
+        int32_t *kv_qend = reinterpret_cast<int32_t *>(ws + L.kv_qend);
+        kv_qend_kernel<<<static_cast<int>(ceil_div(T, 256)), 256, 0, stream>>>(N, T, doc_start, kv_qend);
+        unit_order_kernel<Unit::kQueryTiles><<<1, kDbThreads, 0, stream>>>(win.q_tiles, win, T, tile_lo, ghist,
+                                                                            q_order, 0);
+        unit_order_kernel<Unit::kKeyTiles><<<1, kDbThreads, 0, stream>>>(T, win, T, kv_qend, ghist,
+                                                                          reinterpret_cast<int32_t *>(ws + L.kv_order), 0);
+    } else if (fwd_tile_pairs) {
+        unit_order_kernel<Unit::kQueryPairs><<<1, kDbThreads, 0, stream>>>((win.q_tiles + 1) / 2, win, 2 * T,
+                                                                            tile_lo, ghist, q_order, 1);
+    } else {
+        unit_order_kernel<Unit::kQueryTiles><<<1, kDbThreads, 0, stream>>>(win.q_tiles, win, T, tile_lo, ghist,
+                                                                            q_order, 1);
+    }
     return cudaGetLastError();
 }
 

@@ -10,6 +10,7 @@ namespace uly {
 
 constexpr int kTileM = 128;   // query rows per tile
 constexpr int kTileN = 128;   // keys per tile
+constexpr int kScanBlock = 1024;   // tokens per block of the doc-start scan
 constexpr uint32_t kStatusTimeoutHost = 1u;   // same bit as the device-side timeout flag
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -23,6 +24,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 //   q_order    int32  [T]         query tiles heaviest first (backward, and the
 //                                 forward when its items pair heads); forward with
 //                                 tile-pair items: pairs (2u, 2u+1), heaviest first
+//   block_agg  int32  [nb]        per-block maxima of the doc-start scan (nb = ceil(N/1024))
+//   block_carry int32 [nb]        each block's carry (used when nb > 1024)
 //   scratch    int32  [2T + 2]    histogram for the tile sort (when it does not
 //                                 fit in the sorting CTA's shared memory)
 // backward only (Npad = T * 128):
@@ -31,7 +34,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 //   delta      fp32   [Hl][Npad]  D_i = sum_c dO_ic O_ic (0 on padding rows)
 //   lse2       fp32   [Hl][Npad]  LSE_i * log2(e) (+inf on padding rows)
 struct WsLayout {
-    size_t status, doc_start, tile_lo, q_order, scratch;
+    size_t status, doc_start, tile_lo, q_order, block_agg, block_carry, scratch;
     size_t kv_qend, kv_order, delta, lse2;
     size_t total;
 };
@@ -45,6 +48,8 @@ inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
     L.doc_start = off; off += align256(static_cast<size_t>(N) * 4);
     L.tile_lo = off;   off += align256(static_cast<size_t>(T) * 4);
     L.q_order = off;   off += align256(static_cast<size_t>(T) * 4);
+    L.block_agg = off;   off += align256(static_cast<size_t>(ceil_div(N, kScanBlock)) * 4);
+    L.block_carry = off; off += align256(static_cast<size_t>(ceil_div(N, kScanBlock)) * 4);
     L.scratch = off;   off += align256(static_cast<size_t>(2 * T + 2) * 4);
     if (backward) {
         L.kv_qend = off;  off += align256(static_cast<size_t>(T) * 4);
@@ -70,7 +75,7 @@ inline bool fwd_pairs_heads(int Hl, int Hkvl) { return Hkvl > 0 && (Hl / Hkvl) %
 
 // docbounds.cu: doc_start, tile_lo and the query order (single tiles, or
 // pairs of tiles for a forward with tile-pair items; for the backward also
-// kv_qend and the key-tile order), in one single-CTA launch that lets the next
+// kv_qend and the key-tile order); the forward's last sort lets the attention
 // kernel start early (programmatic dependent launch).
 // The forward's schedule covers query tiles [q_tile0, q_tile0 + q_tiles) and
 // counts only the key tiles kvlo_t .. kvhi_t (the key window); the backward

@@ -222,3 +222,32 @@ def test_fwd_irregular_position_ids(kind, Hl, Hkvl, d):
     ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], pos)
     assert_close("O", bf16_to_f64(o), ro)
     assert_close("LSE", lse.double().cpu().numpy(), rl)
+
+
+def test_fwd_beyond_1024_scan_blocks():
+    """More than 1024 blocks of the document-start scan (N > 1048576), where
+    each block's carry comes from a separate prefix over the block maxima: a
+    document that starts in block 1020 and spans 40 more blocks, and short
+    documents elsewhere; rows sampled across block and tile boundaries."""
+    import long_context_sequence_ulysses_b200 as U
+    N = 1024 * 1100
+    start, long_len = 1020 * 1024 + 7, 40 * 1024 + 300
+    lengths = [4096] * (start // 4096)
+    if start > sum(lengths):
+        lengths.append(start - sum(lengths))
+    lengths.append(long_len)
+    rest = N - sum(lengths)
+    lengths += [4096] * (rest // 4096) + ([rest % 4096] if rest % 4096 else [])
+    lengths = [L for L in lengths if L > 0]
+    assert sum(lengths) == N
+    c = random_case(N, 2, 1, 64, lengths, seed=81, device="cuda")
+    o, lse = _run(c)
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([
+        [start, start + 1, start + 1023, start + long_len - 1, N - 1, 1048575, 1048576],
+        np.arange(1021 * 1024 - 2, 1021 * 1024 + 2), np.arange(1050 * 1024 - 2, 1050 * 1024 + 2),
+        rng.integers(start, start + long_len, 48), rng.integers(0, N, 48)]))
+    ro, rl = oracle.attn_fwd(c["q"].cpu(), c["k"].cpu(), c["v"].cpu(), c["position_ids"].cpu(), rows=rows)
+    rt = torch.from_numpy(rows).cuda()
+    assert_close("O", bf16_to_f64(o[rt]), ro)
+    assert_close("LSE", lse[:, rt].double().cpu().numpy(), rl)
