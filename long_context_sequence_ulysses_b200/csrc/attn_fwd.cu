@@ -95,6 +95,11 @@ struct FwdParams {
     int pair_heads;        // 1: items pair heads (T x Hl/2 items); 0: items pair tiles (ceil(T/2) x Hl)
     int items;
     uint32_t *status;      // [0] status word, [1] work counter (both zeroed before the launch)
+    // 1: each tile's O is staged in its Q buffer (free once the item's last S
+    // has run) and written by TMA bulk stores of whole rows; the Q buffer is
+    // released to the producer by the epilogue, after the store has read it.
+    // 0 (a query window that does not start on a tile): per-thread row stores.
+    int o_tma;
     uint64_t wait_limit_ns;
     uint32_t debug_flags;   // bit 0: CTA 0 waits on a barrier nobody arrives on (tests the timeout path)
 };
@@ -173,7 +178,7 @@ struct FwdCfg {
     static constexpr int OFF_K = 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
-    static constexpr int NBAR = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 2 + 2 + 1 + 1;
+    static constexpr int NBAR = 2 + 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 2 + 2 + 1 + 1 + 2;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 2 * kItemInts * 4 + 1024;   // + item ring, alignment slack
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kTileM, kTileN, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kTileM, D, false, true);
@@ -185,7 +190,8 @@ struct FwdCfg {
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdParams p)
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const FwdParams p)
 {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -195,7 +201,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint8_t *sV = smem + C::OFF_V;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars;                 // [2]
-    uint64_t *q_empty = bars + 2;            // [2] the last S of an item has read Q_x
+    uint64_t *q_empty = bars + 2;            // [2] Q_x is free: its item's last S has read it (or,
+                                             // with o_tma, its epilogue's store has read the O staged there)
     uint64_t *k_full = bars + 4;             // [KST]
     uint64_t *k_empty = k_full + C::KST;
     uint64_t *v_full = k_empty + C::KST;     // [VST]
@@ -207,7 +214,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t *item_empty = item_full + 2;    // [2] item ring slot read by every consumer
     uint64_t *mma_done = item_empty + 2;
     uint64_t *never = mma_done + 1;          // never arrived on (timeout test only)
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(never + 1);
+    uint64_t *o_staged = never + 1;          // [2] every row of tile x's O is staged (o_tma)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(o_staged + 2);
     // two decoded FwdItems, written by the producer, read by every other role
     volatile int *item_ring = reinterpret_cast<volatile int *>(tmem_holder + 4);
 
@@ -225,6 +233,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(&o_done[x], 1);
             mbar_init(&item_full[x], 1);
             mbar_init(&item_empty[x], kItemConsumers);
+            mbar_init(&o_staged[x], 128);
         }
         for (int s = 0; s < C::KST; ++s) {
             mbar_init(&k_full[s], 1);
@@ -420,8 +429,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const bool pvB = have_cur && cur.hasB && cur.nB > 0;
             const bool sA = have_nxt && nxt.nA > 0;
             const bool sB = have_nxt && nxt.hasB && nxt.nB > 0 && nxt.bstart == 0;
+            // With O staged in the Q buffers (o_tma) the next item's Q tiles arrive only
+            // after this item's epilogues, so both last PVs go first.
+            const bool late_q = p.o_tma != 0;
             if (pvA || pvB) ok = mbar_wait_warp(&v_full[sp], up & 1, wc);
-            if (ok && sA) ok = mbar_wait_warp(&k_full[s], u & 1, wc);
+            if (ok && sA && !late_q) ok = mbar_wait_warp(&k_full[s], u & 1, wc);
             if (ok && pvA) {
                 ok = mbar_wait_warp(&p_full[0], (pbase[0] + cur.nA - 1) & 1, wc);
                 if (ok) {
@@ -430,7 +442,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     umma_commit_elect(&o_done[0]);
                 }
             }
-            if (ok && sA) {
+            if (ok && sA && !late_q) {
                 ok = mbar_wait_warp(&q_full[0], qcount[0] & 1, wc);
                 ++qcount[0];
                 if (ok) {
@@ -447,6 +459,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     umma_commit_elect(&o_done[1]);
                 }
             }
+            if (ok && sA && late_q) {
+                ok = mbar_wait_warp(&k_full[s], u & 1, wc);
+                if (ok) ok = mbar_wait_warp(&q_full[0], qcount[0] & 1, wc);
+                ++qcount[0];
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0, s);
+                }
+            }
             if (ok && have_nxt && nxt.hasB && nxt.nB > 0) {
                 ok = mbar_wait_warp(&q_full[1], qcount[1] & 1, wc);
                 ++qcount[1];
@@ -454,7 +475,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (ok && sB) {
                 tc_fence_after();
                 issue_s(1, s);
-                if (nxt.nB == 1) umma_commit_elect(&q_empty[1]);
+                if (!late_q && nxt.nB == 1) umma_commit_elect(&q_empty[1]);
             }
             if (!ok) break;
             if (sA) umma_commit_elect(&k_empty[s]);
@@ -490,7 +511,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (sAj) {
                     tc_fence_after();
                     issue_s(0, sj);
-                    if (j == cur.nA - 1) umma_commit_elect(&q_empty[0]);
+                    if (!p.o_tma && j == cur.nA - 1) umma_commit_elect(&q_empty[0]);
                 }
                 // tile B
                 if (pvBj) {
@@ -502,7 +523,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (sBj) {
                     tc_fence_after();
                     issue_s(1, sj);
-                    if (jb == cur.nB - 1) umma_commit_elect(&q_empty[1]);
+                    if (!p.o_tma && jb == cur.nB - 1) umma_commit_elect(&q_empty[1]);
                 }
                 if (sAj || sBj) umma_commit_elect(&k_empty[sj]);
                 if (pvAj || pvBj) umma_commit_elect(&v_empty[spj]);
@@ -523,6 +544,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float sl2 = p.scale_log2;
         int sbase = 0;      // S tiles of this slot consumed by earlier items
         int ocount = 0;     // items finished by this slot
+        int scount = 0;     // O tiles of this slot staged for a TMA store
         bool ok = true;
         if ((p.debug_flags & 1u) && blockIdx.x == 0 && x == 0) ok = mbar_wait_warp(never, 0, wc);   // runs out
         for (int n = 0; ok; ++n) {
@@ -669,18 +691,58 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tmem_ld32(tO, *reinterpret_cast<uint32_t(*)[32]>(orw));
             }
             tmem_ld_wait();
+            if (p.o_tma) {
+                // Stage the bf16 row in this tile's Q buffer in the TMA box layout (atoms of
+                // AW columns x 128 rows, 16-byte chunks swizzled by the row), then one thread
+                // stores the tile with whole-row writes and hands the buffer back.
+                uint8_t *stage = sQ + x * C::TILE_BYTES;
+                constexpr int kChunks = C::SW / 16;   // 16-byte chunks per row of an atom
+                const int swz = C::SW == 128 ? (r & 7) : ((r >> 1) & 3);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t wv[16];
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t wv[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    wv[e] = pack_bf16x2(__uint_as_float(orw[c * 32 + 2 * e]) * inv_l,
-                                        __uint_as_float(orw[c * 32 + 2 * e + 1]) * inv_l);
-                if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+                    for (int e = 0; e < 16; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(orw[c * 32 + 2 * e]) * inv_l,
+                                            __uint_as_float(orw[c * 32 + 2 * e + 1]) * inv_l);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = c * 32 + e * 8;                 // first of these 8 columns
+                        const int atom = col / C::AW, chunk = (col % C::AW) / 8;
+                        uint4 *dst = reinterpret_cast<uint4 *>(stage + atom * C::ATOM_BYTES + r * C::SW +
+                                                               ((chunk ^ swz) % kChunks) * 16);
+                        *dst = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                    }
+                }
+                fence_async_smem();             // the staged row is visible to the TMA store
+                mbar_arrive(&o_staged[x]);
+                if (r == 0) {
+                    // bounded: if a thread of the tile gave up on a wait, this gives up too
+                    if (mbar_wait(&o_staged[x], scount & 1, wc)) {
+                        const int row0 = (x == 0 ? w.tA : w.tB) * kTileM - p.q_lo;
+#pragma unroll
+                        for (int a = 0; a < C::NA; ++a)
+                            tma_store_3d(&tmO, stage + a * C::ATOM_BYTES, a * C::AW, p.o_head0 + hx, row0);
+                        bulk_commit_group();
+                        bulk_wait_read_all();
+                        mbar_arrive(&q_empty[x]);   // the producer may load the next Q_x
+                    }
+                }
+                ++scount;
+            } else {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t wv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(orw[c * 32 + 2 * e]) * inv_l,
+                                            __uint_as_float(orw[c * 32 + 2 * e + 1]) * inv_l);
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                    }
                 }
             }
             if (valid)
@@ -690,6 +752,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     }
 
+    // the softmax threads that issued bulk stores see them complete before the CTA exits
+    if (warp < 8 && (threadIdx.x & 127) == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -701,7 +765,7 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
 {
     using C = FwdCfg<D>;
     static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
-    alignas(64) CUtensorMap tq, tk, tv;
+    alignas(64) CUtensorMap tq, tk, tv, to;
     const int box = C::AW;
     if (!encode_tmap_3d(&tq, a.q, D, a.Hq_total, a.N, int64_t(D) * 2, int64_t(a.Hq_total) * D * 2, box, kTileM,
                         C::SW) ||
@@ -710,6 +774,13 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
         !encode_tmap_3d(&tv, a.v, D, a.Hkv_total, a.N, int64_t(D) * 2, int64_t(a.Hkv_total) * D * 2, box, kTileN,
                         C::SW))
         return cudaErrorInvalidValue;
+    // O through TMA stores when the query window starts on a tile (coordinates
+    // of a store must not be negative): the map's rows are the window's
+    const bool o_tma = (a.q_lo % kTileM) == 0;
+    if (o_tma && !encode_tmap_3d(&to, a.o, D, a.Ho_total, a.q_hi - a.q_lo, int64_t(D) * 2,
+                                 int64_t(a.Ho_total) * D * 2, box, kTileM, C::SW))
+        return cudaErrorInvalidValue;
+    if (!o_tma) to = tq;   // not read
     FwdParams p;
     p.doc_start = reinterpret_cast<const int32_t *>(a.ws + a.L.doc_start);
     p.tile_lo = reinterpret_cast<const int32_t *>(a.ws + a.L.tile_lo);
@@ -741,6 +812,7 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     p.items = static_cast<int>(items);
     p.wait_limit_ns = a.wait_limit_ns;
     p.debug_flags = a.debug_flags;
+    p.o_tma = o_tma ? 1 : 0;
     static bool attr_set[64] = {};
     static int sm_count[64] = {};
     int dev = 0;
@@ -768,7 +840,7 @@ cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D>, tq, tk, tv, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D>, tq, tk, tv, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
