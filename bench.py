@@ -615,6 +615,13 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
+    if args.workload == "layer" and world == 1:
+        # the layer step alone (projections with the exchanges fused in, attention per rank)
+        out = measure_layer(U, WORKLOADS["llama8b"], dev, args, args.steps, args.warmup)
+        out.update({"metric": METRIC, "unit": "TFLOP/s", "n_gpus": 1, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "bf16", "data": "synthetic"})
+        print(json.dumps(out), flush=True)
+        return
     name = "llama8b" if args.workload == "all" else args.workload
     out = measure(U, WORKLOADS[name], dev, args, args.steps, args.warmup, world, rank, dist, headline=True)
     if args.workload == "all" and world == 1:
@@ -887,9 +894,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="all", choices=["all"] + sorted(WORKLOADS),
+    ap.add_argument("--workload", default="all", choices=["all", "layer"] + sorted(WORKLOADS),
                     help="all (default): llama8b as the headline line, the other workloads in its 'workloads' "
-                         "object; or one workload alone")
+                         "object; one workload alone; or layer: llama8b's layer step with the projections")
     ap.add_argument("--chunks", type=int, default=1,
                     help="multi-GPU forward with the heads in this many chunks (head-chunked Ulysses)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
