@@ -63,6 +63,8 @@ KERNEL_SOURCES = {
     "attn_fwd_kernel": ("attn_fwd.cu", "ptx.cuh", "ulysses_internal.cuh"),
     "attn_bwd_dkdv_kernel": ("attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh"),
     "attn_bwd_dq_kernel": ("attn_bwd.cu", "ptx.cuh", "ulysses_internal.cuh"),
+    "proj_gemm_kernel": ("proj.cu", "ptx.cuh", "ulysses_internal.cuh"),
+    "attn_merge_kernel": ("merge.cu", "ulysses_internal.cuh"),
 }
 
 
@@ -592,7 +594,9 @@ def measure_layer(U, w, dev, args, steps, warmup):
             rec["roofline_" + kind] = {"kernel": name, "bound": "tensor", "achieved": round(ach, 2), "peak": peak,
                                        "peak_source": peak_kind + " burst", "unit": "TFLOP/s",
                                        "frac": round(ach / peak, 4), "frac_of_spec_2250": round(ach / SPEC_BF16_TFLOPS, 4),
-                                       "flop_per_launch": flop, "ms_per_launch": round(avg, 4), "traffic": None}
+                                       "flop_per_launch": flop, "ms_per_launch": round(avg, 4),
+                                       "traffic": lookup_traffic("proj_gemm_kernel",
+                                                                 "layer_qkv" if kind == "gemm_qkv" else "layer_out")}
     fwd_avg, fwd_sum = timed.stats("attn_fwd")
     if fwd_sum:
         rec["attn_fwd_tflops"] = round(fwd_flop / (fwd_sum / steps * 1e-3) / 1e12, 2)
