@@ -41,8 +41,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
-FWD_LAUNCHES = 2   # doc-bounds + the attention kernel
-BWD_LAUNCHES = 4   # doc-bounds + delta, dK/dV and dQ kernels
+
+
+def fwd_launches(n):
+    """Kernels of one forward call over n tokens: the document scan, its carry
+    prefix (only past 2^20 tokens), the fix-up, the work order, the attention."""
+    return 4 + (n > 1 << 20)
+
+
+def bwd_launches(n):
+    """Kernels of one backward call: the document scan, its carry prefix (past
+    2^20 tokens), the fix-up, the key-tile query ends, the two work orders, the
+    delta prep, the dK/dV kernel and the dQ kernel."""
+    return 8 + (n > 1 << 20)
+
+
 # Workloads the default run measures after the headline one, with the steps
 # each times (the million-token step lasts about a second: 3 are enough).
 SUB_WORKLOADS = ("tiny", "long131k", "million", "train", "hybrid_kv2")
@@ -229,7 +242,7 @@ def build_single(U, w, inp, dev, timed, attn_ranks=None):
         # second all-to-all: O back to sequence shards
         timed("relayout", lambda: U.head_to_seq(o_all, P, out=o_seq))
 
-    launches = 3 + FWD_LAUNCHES * len(ranks) + 1 + ((1 + BWD_LAUNCHES * len(ranks) + 3) if w.backward else 0)
+    launches = 3 + fwd_launches(w.N) * len(ranks) + 1 + ((1 + bwd_launches(w.N) * len(ranks) + 3) if w.backward else 0)
     return step, launches, ws
 
 
@@ -248,7 +261,7 @@ def build_hybrid(U, w, inp, dev, timed):
     def step():
         hybrid.forward(inp["q"], inp["k"], inp["v"], pos, w.P, w.ulysses, plan=plan, out=o_seq, timed=timed)
 
-    return step, 3 + FWD_LAUNCHES * n_steps + n_ranks + 1, plan.ws
+    return step, 3 + fwd_launches(w.N) * n_steps + n_ranks + 1, plan.ws
 
 
 def build_fused(U, w, inp, dev):
@@ -273,7 +286,7 @@ def build_fused(U, w, inp, dev):
                 U.attn_bwd_fused(q_seq, k_seq, v_seq, o_seq, do_seq, lse_all[r * Hl:(r + 1) * Hl], pos, P, r,
                                  dq=dq_seq, dk=dk_seq, dv=dv_seq, ws=ws)
 
-    return step, FWD_LAUNCHES * P + (BWD_LAUNCHES * P if w.backward else 0), ws
+    return step, fwd_launches(w.N) * P + (bwd_launches(w.N) * P if w.backward else 0), ws
 
 
 def time_fused(U, w, inp, dev, steps, total_flop):
@@ -335,7 +348,7 @@ def build_multi(U, w, inp, dev, timed, G, rank, chunks=1):
                                                                                     chunks))
             o_loc.copy_(o)
 
-        return step, chunks * (3 + FWD_LAUNCHES + 1), ws
+        return step, chunks * (3 + fwd_launches(w.N) + 1), ws
 
     def step():
         udist.gather_position_ids(pos_loc, out=pos)
@@ -351,7 +364,7 @@ def build_multi(U, w, inp, dev, timed, G, rank, chunks=1):
             timed("exchange", lambda: udist.head_to_seq(dv_h, recv=rdv, out=dv_loc))
         timed("exchange", lambda: udist.head_to_seq(o_head, recv=ro, out=o_loc))
 
-    launches = 3 + FWD_LAUNCHES + 1 + ((1 + BWD_LAUNCHES + 3) if w.backward else 0)
+    launches = 3 + fwd_launches(w.N) + 1 + ((1 + bwd_launches(w.N) + 3) if w.backward else 0)
     return step, launches, ws
 
 
@@ -585,7 +598,7 @@ def measure_layer(U, w, dev, args, steps, warmup):
                                         "step": "qkv_proj into every rank's head slice (fused first exchange); "
                                                 "attn_fwd per rank; out_proj from the head slices (fused second "
                                                 "exchange)", "weights": "random-init, N(0, 1/hidden), seeded"},
-           "clocks": clocks, "gpu_launches": (2 + FWD_LAUNCHES * P) * steps}
+           "clocks": clocks, "gpu_launches": (2 + fwd_launches(w.N) * P) * steps}
     for kind, flop, name in (("gemm_qkv", qkv_flop, "qkv_proj (proj_gemm_kernel<256>)"),
                              ("gemm_out", out_flop, "out_proj (proj_gemm_kernel<256>)")):
         avg, _ = timed.stats(kind)
@@ -649,7 +662,7 @@ def run_gpu(args):
 
 def run_e2e_pipelined(U, w, inp, args, dev):
     from cuda.bindings import runtime as cudart
-    P, N, d, Hl, H = w.P, w.N, w.d, w.Hl, w.H
+    P, N, d, Hl, H, Hkvl, Hkv = w.P, w.N, w.d, w.Hl, w.H, w.Hkvl, w.Hkv
     pin = lambda t: t.cpu().pin_memory()
     hq, hk, hv, hpos = pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), pin(inp["position_ids"])
     ho = torch.empty_like(hq).pin_memory()
@@ -660,7 +673,8 @@ def run_e2e_pipelined(U, w, inp, args, dev):
     lse_all = torch.empty((H, N), dtype=torch.float32, device=dev)
     ws = torch.empty(U.workspace_bytes(N, Hl, w.Hkvl, d, False), dtype=torch.uint8, device=dev)
     s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    row, cols = H * d * 2, Hl * d * 2            # bytes per token row; bytes of one rank's heads in it
+    row, cols = H * d * 2, Hl * d * 2            # bytes per token row of Q / O; one rank's heads in it
+    krow, kcols = Hkv * d * 2, Hkvl * d * 2      # the same for K and V
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2 + hpos.numel() * 4
     d2h = ho.numel() * 2 + hlse.numel() * 4
     ev_in = [torch.cuda.Event() for _ in range(P)]
@@ -669,8 +683,10 @@ def run_e2e_pipelined(U, w, inp, args, dev):
     ev_done.record(s_out)
     H2D, D2H = cudart.cudaMemcpyKind.cudaMemcpyHostToDevice, cudart.cudaMemcpyKind.cudaMemcpyDeviceToHost
 
-    def copy2d(dst, src, kind, stream):
-        err, = cudart.cudaMemcpy2DAsync(dst, row, src, row, cols, N, kind, cudart.cudaStream_t(stream.cuda_stream))
+    def copy2d(dst, src, kind, stream, pitch=None, width=None):
+        pitch, width = pitch or row, width or cols
+        err, = cudart.cudaMemcpy2DAsync(dst, pitch, src, pitch, width, N, kind,
+                                        cudart.cudaStream_t(stream.cuda_stream))
         if err != cudart.cudaError_t.cudaSuccess:
             raise RuntimeError(f"cudaMemcpy2DAsync: {err}")
 
@@ -678,9 +694,10 @@ def run_e2e_pipelined(U, w, inp, args, dev):
         s_in.wait_event(ev_done)                  # the previous step has read everything back
         with torch.cuda.stream(s_in):
             gpos.copy_(hpos, non_blocking=True)
-            gk.copy_(hk, non_blocking=True)
-            gv.copy_(hv, non_blocking=True)
             for r in range(P):
+                # rank r's query heads and KV heads: one pitched copy each
+                copy2d(gk.data_ptr() + r * kcols, hk.data_ptr() + r * kcols, H2D, s_in, krow, kcols)
+                copy2d(gv.data_ptr() + r * kcols, hv.data_ptr() + r * kcols, H2D, s_in, krow, kcols)
                 copy2d(gq.data_ptr() + r * cols, hq.data_ptr() + r * cols, H2D, s_in)
                 ev_in[r].record(s_in)
         with torch.cuda.stream(s_cmp):
@@ -711,7 +728,7 @@ def run_e2e_pipelined(U, w, inp, args, dev):
     return {"value": round((fwd_flop + bwd_flop) / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": args.e2e_steps,
-            "path": "pinned host -> device copies (K, V, ids, then each rank's query heads as one pitched copy), "
+            "path": "pinned host -> device copies (ids, then each rank's K, V and query heads as pitched copies), "
                     "attn_fwd_fused per rank as its heads arrive, each rank's O columns and LSE back on a third "
                     "stream"}
 
@@ -719,8 +736,8 @@ def run_e2e_pipelined(U, w, inp, args, dev):
 def run_e2e(U, w, inp, args, dev):
     """The step through the public API from pinned HOST buffers, host<->device
     copies inside the timed region. A forward-only workload runs as a
-    three-stream pipeline over the emulated ranks: K, V and the position ids
-    are copied first, then rank r's query heads (one pitched copy of those
+    three-stream pipeline over the emulated ranks: the position ids first,
+    then rank by rank its KV heads and query heads (pitched copies of those
     columns of every token row); rank r's fused attention (which reads its
     heads straight from the sequence layout) starts as soon as its heads have
     arrived, and its O columns and LSE rows go back to the host on a third

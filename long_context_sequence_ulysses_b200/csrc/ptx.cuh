@@ -48,18 +48,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-// Potentially blocking probe: the thread may sleep up to about `hint_ns`
-// (a suspend-time hint) waiting for the phase before returning false, so a
-// waiting warp does not take issue slots from the warps that compute.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns = 20000u)
+// Potentially blocking probe: the thread may be suspended for a
+// hardware-chosen time waiting for the phase before returning false, so a
+// waiting warp does not take issue slots from the warps that compute. (An
+// explicit suspend-time hint of 2 or 20 us measured 0.5 % slower on the
+// forward than leaving the choice to the hardware.)
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
