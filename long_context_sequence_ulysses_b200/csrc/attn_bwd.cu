@@ -48,8 +48,9 @@ namespace {
 // phases. Each part writes its bf16 results to the first half of its own
 // columns, so no part overwrites columns another still has to read; the TS
 // MMAs find K step kk (16 rows, 8 packed columns) at pcol(kk).
-// All exponentials go to the SFU here: moving part of them to the FMA-pipe
-// polynomial (as the forward does) measured slower in both kernels.
+// All exponentials go to the SFU here: moving 1 or 2 of every 8 pairs to the
+// FMA-pipe polynomial (as the forward does) measured no faster in either
+// kernel (the special-function unit is not what bounds them).
 constexpr int kParts = 4;
 constexpr int kPartCols = kTileN / kParts;
 constexpr int kBwdThreads = 128 + kParts * 128;
