@@ -17,10 +17,16 @@
 //     see the key tile and, for each, the query heads of the GQA group (heads
 //     inner: CTAs of neighbouring key tiles then read the same Q / dO tiles a
 //     few steps apart, while they are still in L2):
-//       S^T = K Q^T, dP^T = V dO^T       (SS MMA, M = keys, N = queries)
+//       S^T = K Q^T - LSE / scale, dP^T = V dO^T - D
+//                                         (SS MMA, M = keys, N = queries)
 //       P^T, dS^T -> bf16 into the first 64 columns of S^T / dP^T in TMEM
 //       dV += P^T dO, dK += dS^T Q      (TS MMA, dO / Q read MN-major)
-//     so the group reduction happens in the accumulator. The element-wise
+//     so the group reduction happens in the accumulator. The per-query terms
+//     enter S^T and dP^T as one extra 16-wide K step (a column of ones
+//     against each query's term split into hi and lo bf16 halves, exact to
+//     about 2^-17 relative): the element-wise threads then read no per-query
+//     values at all (as broadcast shared-memory loads, those took 41 % of the
+//     shared-memory load bandwidth). The element-wise
 //     step runs in two phases so that the tensor core always has work: once
 //     P^T(i) is stored, dV(i) and S^T(i+1) run while dS^T(i) is computed
 //     (from the bf16 P^T kept in registers); once dS^T(i) is stored, dK(i)
@@ -87,14 +93,18 @@ struct BwdCfg {
     static constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, false, true);
     static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
-    // dK/dV kernel shared memory: K, V, then NST stages of {Q, dO}, then
-    // NST stages of {lse2 row, delta row} (512 bytes each), then barriers.
+    // dK/dV kernel shared memory: K, V, then NST stages of {Q, dO}, then NST
+    // stages of the extra K-step blocks {QB, DB} (128 rows x 16 bf16, 32-byte
+    // swizzle), the constant block of ones, then barriers.
+    static constexpr int XB_BYTES = kTileM * kXStepBytes;
     static constexpr int KV_OFF_K = 0;
     static constexpr int KV_OFF_V = TILE_BYTES;
     static constexpr int KV_OFF_Q = 2 * TILE_BYTES;
     static constexpr int KV_OFF_DO = KV_OFF_Q + NST * TILE_BYTES;
-    static constexpr int KV_OFF_ROW = KV_OFF_DO + NST * TILE_BYTES;
-    static constexpr int KV_OFF_BAR = KV_OFF_ROW + NST * 2 * 512;
+    static constexpr int KV_OFF_QB = KV_OFF_DO + NST * TILE_BYTES;
+    static constexpr int KV_OFF_DB = KV_OFF_QB + NST * XB_BYTES;
+    static constexpr int KV_OFF_ONES = KV_OFF_DB + NST * XB_BYTES;
+    static constexpr int KV_OFF_BAR = KV_OFF_ONES + XB_BYTES;
     static constexpr int KV_SMEM = KV_OFF_BAR + 16 * 8 + 16 + 1024;
     // dQ kernel shared memory: Q, dO, then QKST stages of K and QVST of V,
     // then barriers. S runs two key tiles ahead of dQ, so a K tile is needed
@@ -126,14 +136,36 @@ __device__ __forceinline__ float dot8_bf16(const uint4 &a, const uint4 &b)
     return acc;
 }
 
+// Two bf16 values whose sum is v to about 2^-17 relative: v's rounding and
+// the rounding of what it left over.
+__device__ __forceinline__ uint32_t bf16_hi_lo(float v)
+{
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float rest = isinf(v) ? 0.f : v - __bfloat162float(hi);
+    return pack_bf16x2(__bfloat162float(hi), rest);
+}
+
 // D_i = sum_c dO_ic O_ic and -LSE_i * log2(e), one warp per (head, padded row).
+// For the dK/dV kernel the same two terms also go, as hi/lo bf16 pairs, into
+// an extra K step of its products: row (i, h) of qb holds -LSE_i / scale
+// (S^T + that, times scale*log2(e), is the exponent of P^T), row (i, h) of db
+// holds -D_i (dP^T + that is dP^T - D); a padding row gets -inf and 0. The
+// first 128 threads also write the block of ones the key side multiplies
+// them with.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
                                                       const __nv_bfloat16 *__restrict__ dout,
                                                       const float *__restrict__ lse, float *__restrict__ delta,
-                                                      float *__restrict__ lse2, int N, int Npad, int Hl,
-                                                      int Hq_total, int q_head0)
+                                                      float *__restrict__ lse2, uint4 *__restrict__ qb,
+                                                      uint4 *__restrict__ db, uint4 *__restrict__ ones,
+                                                      float inv_scale, int N, int Npad, int Hl, int Hq_total,
+                                                      int q_head0)
 {
+    if (blockIdx.x == 0 && threadIdx.x < kTileM) {
+        const uint32_t one2 = pack_bf16x2(1.f, 1.f);
+        ones[2 * threadIdx.x] = make_uint4(one2, 0u, 0u, 0u);
+        ones[2 * threadIdx.x + 1] = make_uint4(0u, 0u, 0u, 0u);
+    }
     const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (w >= static_cast<int64_t>(Hl) * Npad) return;
@@ -149,17 +181,16 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
+        const float lse_i = i < N ? lse[static_cast<int64_t>(h) * N + i] : CUDART_INF_F;
         delta[w] = i < N ? acc : 0.f;
-        lse2[w] = i < N ? -lse[static_cast<int64_t>(h) * N + i] * kLog2e : -CUDART_INF_F;
+        lse2[w] = i < N ? -lse_i * kLog2e : -CUDART_INF_F;
+        // rows [Npad][Hl] of 16 bf16: the extra K step's operand tiles load like Q's
+        const int64_t xr = (static_cast<int64_t>(i) * Hl + h) * 2;
+        qb[xr] = make_uint4(bf16_hi_lo(i < N ? -lse_i * inv_scale : -CUDART_INF_F), 0u, 0u, 0u);
+        qb[xr + 1] = make_uint4(0u, 0u, 0u, 0u);
+        db[xr] = make_uint4(bf16_hi_lo(i < N ? -acc : 0.f), 0u, 0u, 0u);
+        db[xr + 1] = make_uint4(0u, 0u, 0u, 0u);
     }
-}
-
-__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
 }
 
 // Column of the bf16 operand packed in tensor memory for K step kk (16 rows
@@ -203,7 +234,8 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                         const BwdParams p)
+                         const __grid_constant__ CUtensorMap tmQB, const __grid_constant__ CUtensorMap tmDB,
+                         const __grid_constant__ CUtensorMap tmOnes, const BwdParams p)
 {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -212,7 +244,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *sV = smem + C::KV_OFF_V;
     uint8_t *sQ = smem + C::KV_OFF_Q;
     uint8_t *sDO = smem + C::KV_OFF_DO;
-    float *sRow = reinterpret_cast<float *>(smem + C::KV_OFF_ROW);   // [NST][2][128]: lse2, delta
+    uint8_t *sQB = smem + C::KV_OFF_QB;
+    uint8_t *sDB = smem + C::KV_OFF_DB;
+    uint8_t *sOnes = smem + C::KV_OFF_ONES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::KV_OFF_BAR);
     uint64_t *kv_full = bars;
     uint64_t *qdo_full = bars + 1;            // [NST]
@@ -261,9 +295,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full, 2 * C::TILE_BYTES);
+            mbar_arrive_expect_tx(kv_full, 2 * C::TILE_BYTES + C::XB_BYTES);
             tma_tile<D>(&tmK, sK, kv_full, p.kv_head0 + kvh, t * kTileN);
             tma_tile<D>(&tmV, sV, kv_full, p.kv_head0 + kvh, t * kTileN);
+            tma_load_3d(sOnes, &tmOnes, kv_full, 0, 0, 0);
             int last_use[C::NST];
 #pragma unroll
             for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
@@ -272,12 +307,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int h = kvh * G + it % G;
                 const int qt = qt0 + it / G;
                 if (u > 0 && !mbar_wait(&qdo_empty[s], (u - 1) & 1, wc)) break;
-                mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES + 2 * 512);
+                mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES + 2 * C::XB_BYTES);
                 tma_tile<D>(&tmQ, sQ + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
                 tma_tile<D>(&tmDO, sDO + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
-                const int64_t roff = static_cast<int64_t>(h) * p.Npad + static_cast<int64_t>(qt) * kTileM;
-                bulk_load(sRow + (s * 2 + 0) * 128, p.lse2 + roff, 512, &qdo_full[s]);
-                bulk_load(sRow + (s * 2 + 1) * 128, p.delta + roff, 512, &qdo_full[s]);
+                tma_load_3d(sQB + s * C::XB_BYTES, &tmQB, &qdo_full[s], 0, h, qt * kTileM);
+                tma_load_3d(sDB + s * C::XB_BYTES, &tmDB, &qdo_full[s], 0, h, qt * kTileM);
                 last_use[s] = u;
             }
             WaitCtx drain{p.wait_limit_ns, p.status, false};
@@ -289,19 +323,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ------------------------------------------------ MMA issuer
         {   // the whole warp runs the loop; elect.sync picks the issuing lane
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
+            // the extra K step: a column of ones (in pairs) against each query's hi/lo terms
+            const uint64_t d_ones = smem_desc(smem_u32(sOnes), 16, 8 * kXStepBytes, kSwizzle32);
             bool ok = mbar_wait_warp(kv_full, 0, wc);
-            auto issue_s = [&](int st) {   // S^T = K Q^T for the query tile in stage st
+            auto issue_s = [&](int st) {   // S^T = K Q^T - LSE / scale for the query tile in stage st
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     umma_ss_elect(tbase + C::T_S, kmajor_desc<D>(aK, kk), kmajor_desc<D>(aQ + st * C::TILE_BYTES, kk),
                                   C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_ss_elect(tbase + C::T_S, d_ones,
+                              smem_desc(smem_u32(sQB + st * C::XB_BYTES), 16, 8 * kXStepBytes, kSwizzle32),
+                              C::IDESC_SS, 1u);
                 umma_commit_elect(s_full);
             };
-            auto issue_dp = [&](int st) {   // dP^T = V dO^T
+            auto issue_dp = [&](int st) {   // dP^T = V dO^T - D
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     umma_ss_elect(tbase + C::T_DP, kmajor_desc<D>(aV, kk), kmajor_desc<D>(aDO + st * C::TILE_BYTES, kk),
                                   C::IDESC_SS, kk > 0 ? 1u : 0u);
+                umma_ss_elect(tbase + C::T_DP, d_ones,
+                              smem_desc(smem_u32(sDB + st * C::XB_BYTES), 16, 8 * kXStepBytes, kSwizzle32),
+                              C::IDESC_SS, 1u);
                 umma_commit_elect(dp_full);
             };
             if (ok && n_it > 0) {
@@ -362,32 +404,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t col = static_cast<uint32_t>(part * kPartCols);   // this part's columns in S^T / dP^T
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
-            const int s = it % C::NST, u = it / C::NST;
             const int q0 = (qt0 + it / G) * kTileM + part * kPartCols;   // first query of this part
-            // warp-uniform waits: the tcgen05.ld below needs the whole warp converged
+            // warp-uniform wait: the tcgen05.ld below needs the whole warp converged
             if (!mbar_wait_warp(s_full, it & 1, wc)) { ok = false; break; }
-            if (!mbar_wait_warp(&qdo_full[s], u & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const float *rl = sRow + (s * 2 + 0) * 128 + part * kPartCols;   // -lse2 of this part's queries
-            const float *rd = sRow + (s * 2 + 1) * 128 + part * kPartCols;   // delta of this part's queries
             const bool any_mask = __any_sync(0xffffffffu, (q0 < j) || (q0 + kPartCols - 1 >= dend));
-            // phase 1: P^T = exp2(S^T * scale*log2(e) - LSE*log2(e)), bf16 into S^T's columns;
-            // the per-query values are fetched as float4 before waiting for the tensor-memory load
+            // phase 1: P^T = exp2((S^T - LSE / scale) * scale*log2(e)), bf16 into S^T's
+            // columns (the products' extra K step has already subtracted LSE / scale)
             float pf[kPartCols];   // P^T in fp32: dS is formed from it, rounded once
             {
                 uint32_t pp[kPartCols / 2];
                 uint32_t sr[kPartCols];
                 tmem_ld32(tbase + C::T_S + lane_off + col, sr);
-                float4 nl[kPartCols / 4];
-#pragma unroll
-                for (int v = 0; v < kPartCols / 4; ++v) nl[v] = *reinterpret_cast<const float4 *>(rl + 4 * v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < kPartCols / 2; ++e) {
-                    const float4 &n4 = nl[e >> 1];
-                    const float a0 = (e & 1) ? n4.z : n4.x, a1 = (e & 1) ? n4.w : n4.y;
                     float x0, x1;
-                    fma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2, a0, a1);
+                    mul2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), sl2, sl2);
                     if (any_mask) {
                         const int qi = q0 + 2 * e;
                         if (qi < j || qi >= dend) x0 = -CUDART_INF_F;
@@ -402,24 +435,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_ready);
-            // phase 2: dS^T = P^T (dP^T - D) from the fp32 P^T, bf16 into dP^T's columns
+            // phase 2: dS^T = P^T (dP^T - D) from the fp32 P^T (the products' extra K step
+            // has already subtracted D), bf16 into dP^T's columns
             if (!mbar_wait_warp(dp_full, it & 1, wc)) { ok = false; break; }
             tc_fence_after();
             {
                 uint32_t dr[kPartCols];
                 tmem_ld32(tbase + C::T_DP + lane_off + col, dr);
-                float4 dl[kPartCols / 4];
-#pragma unroll
-                for (int v = 0; v < kPartCols / 4; ++v) dl[v] = *reinterpret_cast<const float4 *>(rd + 4 * v);
                 tmem_ld_wait();
                 uint32_t dd[kPartCols / 2];
 #pragma unroll
                 for (int e = 0; e < kPartCols / 2; ++e) {
-                    const float4 &d4 = dl[e >> 1];
-                    const float b0 = (e & 1) ? d4.z : d4.x, b1 = (e & 1) ? d4.w : d4.y;
-                    float t0, t1, d0, d1;
-                    sub2(t0, t1, __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]), b0, b1);
-                    mul2(d0, d1, pf[2 * e], pf[2 * e + 1], t0, t1);
+                    float d0, d1;
+                    mul2(d0, d1, pf[2 * e], pf[2 * e + 1], __uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]));
                     dd[e] = pack_bf16x2(d0, d1);
                 }
                 tmem_st16(tbase + C::T_DP + lane_off + col, dd);   // dS^T
@@ -733,6 +761,13 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
         !encode_tmap_3d(&tk, a.k, D, a.Hkv_total, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW) ||
         !encode_tmap_3d(&tv, a.v, D, a.Hkv_total, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW))
         return cudaErrorInvalidValue;
+    // the dK/dV kernel's extra K-step operands: rows [Npad][Hl][16] bf16, and the block of ones
+    alignas(64) CUtensorMap tqb, tdb, tones;
+    const int64_t xs = int64_t(a.Hl) * kXStepBytes;
+    if (!encode_tmap_3d(&tqb, a.ws + a.L.qb, 16, a.Hl, Npad, kXStepBytes, xs, 16, kTileM, kXStepBytes) ||
+        !encode_tmap_3d(&tdb, a.ws + a.L.db, 16, a.Hl, Npad, kXStepBytes, xs, 16, kTileM, kXStepBytes) ||
+        !encode_tmap_3d(&tones, a.ws + a.L.ones, 16, 1, kTileM, kXStepBytes, kXStepBytes, 16, kTileM, kXStepBytes))
+        return cudaErrorInvalidValue;
     BwdParams p;
     p.doc_start = reinterpret_cast<const int32_t *>(a.ws + a.L.doc_start);
     p.tile_lo = reinterpret_cast<const int32_t *>(a.ws + a.L.tile_lo);
@@ -763,14 +798,15 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     const int64_t prep_threads = int64_t(a.Hl) * Npad * 32;
     bwd_prep_kernel<D><<<static_cast<unsigned>(ceil_div(prep_threads, 256)), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, delta, lse2,
-        p.N, Npad, a.Hl, a.Hq_total, a.q_head0);
+        reinterpret_cast<uint4 *>(a.ws + a.L.qb), reinterpret_cast<uint4 *>(a.ws + a.L.db),
+        reinterpret_cast<uint4 *>(a.ws + a.L.ones), 1.f / a.scale, p.N, Npad, a.Hl, a.Hq_total, a.q_head0);
     static bool kv_attr[64] = {}, q_attr[64] = {};
     cudaError_t e = set_smem(attn_bwd_dkdv_kernel<D>, C::KV_SMEM, kv_attr);
     if (e != cudaSuccess) return e;
     e = set_smem(attn_bwd_dq_kernel<D>, C::Q_SMEM, q_attr);
     if (e != cudaSuccess) return e;
     attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(int64_t(T) * a.Hkvl), kBwdThreads, C::KV_SMEM, stream>>>(
-        tq, tk, tv, tdo, p);
+        tq, tk, tv, tdo, tqb, tdb, tones, p);
     attn_bwd_dq_kernel<D><<<static_cast<unsigned>(int64_t(T) * a.Hl), kBwdThreads, C::Q_SMEM, stream>>>(
         tq, tk, tv, tdo, p);
     return cudaGetLastError();

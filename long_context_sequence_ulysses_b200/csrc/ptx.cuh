@@ -352,6 +352,7 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 //   bits 61-63 swizzle mode: 0 none, 2 = 128-byte, 4 = 64-byte, 6 = 32-byte
 constexpr uint32_t kSwizzle128 = 2;
 constexpr uint32_t kSwizzle64 = 4;
+constexpr uint32_t kSwizzle32 = 6;
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t swizzle_mode)

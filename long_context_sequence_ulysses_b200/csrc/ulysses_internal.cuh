@@ -33,9 +33,14 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 //   kv_order   int32  [T]         key tiles, heaviest first
 //   delta      fp32   [Hl][Npad]  D_i = sum_c dO_ic O_ic (0 on padding rows)
 //   lse2       fp32   [Hl][Npad]  LSE_i * log2(e) (+inf on padding rows)
+// Bytes of one row of an extra 16-element (bf16) K step of the backward's
+// S^T and dP^T products.
+constexpr int kXStepBytes = 32;
+
 struct WsLayout {
     size_t status, doc_start, tile_lo, q_order, block_agg, block_carry, scratch;
     size_t kv_qend, kv_order, delta, lse2;
+    size_t qb, db, ones;   // backward: per-query terms as an extra K step (see attn_bwd.cu)
     size_t total;
 };
 
@@ -56,8 +61,11 @@ inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
         L.kv_order = off; off += align256(static_cast<size_t>(T) * 4);
         L.delta = off;    off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
         L.lse2 = off;     off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
+        L.qb = off;       off += align256(static_cast<size_t>(T) * kTileM * Hl * kXStepBytes);
+        L.db = off;       off += align256(static_cast<size_t>(T) * kTileM * Hl * kXStepBytes);
+        L.ones = off;     off += align256(static_cast<size_t>(kTileM) * kXStepBytes);
     } else {
-        L.kv_qend = L.kv_order = L.delta = L.lse2 = 0;
+        L.kv_qend = L.kv_order = L.delta = L.lse2 = L.qb = L.db = L.ones = 0;
     }
     L.total = off;
     return L;
