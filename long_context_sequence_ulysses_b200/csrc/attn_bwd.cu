@@ -26,16 +26,16 @@
 //     against each query's term split into hi and lo bf16 halves, exact to
 //     about 2^-17 relative): the element-wise threads then read no per-query
 //     values at all (as broadcast shared-memory loads, those took 41 % of the
-//     shared-memory load bandwidth). The element-wise
-//     step runs in two phases so that the tensor core always has work: once
-//     P^T(i) is stored, dV(i) and S^T(i+1) run while dS^T(i) is computed
-//     (from the bf16 P^T kept in registers); once dS^T(i) is stored, dK(i)
-//     and dP^T(i+1) run while P^T(i+1) is computed.
+//     shared-memory load bandwidth).
+//     The element-wise step runs in two phases so that the tensor core always
+//     has work: once P^T(i) is stored, dV(i) and S^T(i+1) run while dS^T(i)
+//     is computed (from the fp32 P^T kept in registers); once dS^T(i) is
+//     stored, dK(i) and dP^T(i+1) run while P^T(i+1) is computed.
 //  3. dQ: one CTA per (query tile, head) loops over its key tiles:
 //       S = Q K^T, dP = dO V^T -> dS (bf16, into S's columns) -> dQ += dS K.
 //     S has two buffers (the second in the columns the dQ accumulator leaves
 //     free) and runs two key tiles ahead: P is formed while dP is computed,
-//     and dQ, the next dP and the S after next run while the element-wise
+//     and the next dP, dQ and the S after next run while the element-wise
 //     step of the following tile proceeds.
 #include "ptx.cuh"
 #include "ulysses_internal.cuh"
@@ -629,14 +629,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int s = j % C::QKST;
                 if (!mbar_wait_warp(ds_full, j & 1, wc)) { ok = false; break; }
                 tc_fence_after();
+                // dP(j+1) first: it overwrites only dP(j), which the element-wise step
+                // of j has read, and the next step's phase 1 then finds it done
+                if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
 #pragma unroll
                 for (int kk = 0; kk < kTileN / 16; ++kk)
                     umma_ts_elect(tbase + C::T_ACC0, sbuf(j) + pcol(kk), mnmajor_desc<D>(aK + s * C::TILE_BYTES, kk),
                                   C::IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);   // dQ += dS K
                 umma_commit_elect(&k_empty[s]);
-                // dP(j+1) overwrites dP(j), read by the element-wise step of j;
                 // S(j+2) overwrites dS(j), read by the products just issued
-                if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
                 if (j + 2 < n_kv && !issue_s(j + 2)) { ok = false; break; }
             }
             if (ok) umma_commit_elect(acc_done);
