@@ -24,7 +24,8 @@
 //     so the group reduction happens in the accumulator. The per-query terms
 //     enter S^T and dP^T as one extra 16-wide K step (a column of ones
 //     against each query's term split into hi and lo bf16 halves, exact to
-//     about 2^-17 relative): the element-wise threads then read no per-query
+//     about 2^-17 relative; the producer warp builds those operand tiles from
+//     4 bytes per query): the element-wise threads then read no per-query
 //     values at all (as broadcast shared-memory loads, those took 41 % of the
 //     shared-memory load bandwidth).
 //     The element-wise step runs in two phases so that the tensor core always
@@ -72,6 +73,8 @@ struct BwdParams {
     const int32_t *kv_order;
     const float *delta;   // [Hl][Npad]
     const float *lse2;    // [Hl][Npad]: -LSE * log2(e) (-inf on padding rows)
+    const uint32_t *qx;   // [Hl][Npad]: -LSE / scale as a hi/lo bf16 pair (the dK/dV kernel's extra K step)
+    const uint32_t *dx;   // [Hl][Npad]: -D as a hi/lo bf16 pair
     __nv_bfloat16 *dq, *dk, *dv;
     int N, Npad, T, Hl, Hkvl;
     int Hq_total, Hkv_total;   // heads per token row of the q / kv-side buffers
@@ -147,17 +150,16 @@ __device__ __forceinline__ uint32_t bf16_hi_lo(float v)
 
 // D_i = sum_c dO_ic O_ic and -LSE_i * log2(e), one warp per (head, padded row).
 // For the dK/dV kernel the same two terms also go, as hi/lo bf16 pairs, into
-// an extra K step of its products: row (i, h) of qb holds -LSE_i / scale
-// (S^T + that, times scale*log2(e), is the exponent of P^T), row (i, h) of db
-// holds -D_i (dP^T + that is dP^T - D); a padding row gets -inf and 0. The
-// first 128 threads also write the block of ones the key side multiplies
-// them with.
+// an extra K step of its products: qx[h][i] holds -LSE_i / scale (S^T + that,
+// times scale*log2(e), is the exponent of P^T), dx[h][i] holds -D_i (dP^T +
+// that is dP^T - D); a padding row gets -inf and 0. The first 128 threads
+// also write the block of ones the key side multiplies them with.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
                                                       const __nv_bfloat16 *__restrict__ dout,
                                                       const float *__restrict__ lse, float *__restrict__ delta,
-                                                      float *__restrict__ lse2, uint4 *__restrict__ qb,
-                                                      uint4 *__restrict__ db, uint4 *__restrict__ ones,
+                                                      float *__restrict__ lse2, uint32_t *__restrict__ qx,
+                                                      uint32_t *__restrict__ dx, uint4 *__restrict__ ones,
                                                       float inv_scale, int N, int Npad, int Hl, int Hq_total,
                                                       int q_head0)
 {
@@ -184,12 +186,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
         const float lse_i = i < N ? lse[static_cast<int64_t>(h) * N + i] : CUDART_INF_F;
         delta[w] = i < N ? acc : 0.f;
         lse2[w] = i < N ? -lse_i * kLog2e : -CUDART_INF_F;
-        // rows [Npad][Hl] of 16 bf16: the extra K step's operand tiles load like Q's
-        const int64_t xr = (static_cast<int64_t>(i) * Hl + h) * 2;
-        qb[xr] = make_uint4(bf16_hi_lo(i < N ? -lse_i * inv_scale : -CUDART_INF_F), 0u, 0u, 0u);
-        qb[xr + 1] = make_uint4(0u, 0u, 0u, 0u);
-        db[xr] = make_uint4(bf16_hi_lo(i < N ? -acc : 0.f), 0u, 0u, 0u);
-        db[xr + 1] = make_uint4(0u, 0u, 0u, 0u);
+        qx[w] = bf16_hi_lo(i < N ? -lse_i * inv_scale : -CUDART_INF_F);
+        dx[w] = bf16_hi_lo(i < N ? -acc : 0.f);
     }
 }
 
@@ -234,7 +232,6 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                         const __grid_constant__ CUtensorMap tmQB, const __grid_constant__ CUtensorMap tmDB,
                          const __grid_constant__ CUtensorMap tmOnes, const BwdParams p)
 {
     using C = BwdCfg<D>;
@@ -271,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < C::NST; ++s) {
-            mbar_init(&qdo_full[s], 1);
+            mbar_init(&qdo_full[s], 2);   // the copies' bytes and the producer warp's extra-step tiles
             mbar_init(&qdo_empty[s], 1);
         }
         mbar_init(s_full, 1);
@@ -293,27 +290,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     WaitCtx wc{p.wait_limit_ns, p.status, *reinterpret_cast<volatile uint32_t *>(p.status) != 0u};
 
     if (warp == 0) {
-        // ------------------------------------------------ producer
+        // ------------------------------------------------ producer: lane 0 issues the copies; the
+        // whole warp builds each stage's extra K-step tiles (128 rows x 16 bf16, 32-byte
+        // swizzle: a row's first 16 bytes sit in chunk (row >> 2) & 1) from the compact
+        // per-query terms. Only the first 16 bytes of a row change; the rest stay zero.
         if (lane == 0) {
             mbar_arrive_expect_tx(kv_full, 2 * C::TILE_BYTES + C::XB_BYTES);
             tma_tile<D>(&tmK, sK, kv_full, p.kv_head0 + kvh, t * kTileN);
             tma_tile<D>(&tmV, sV, kv_full, p.kv_head0 + kvh, t * kTileN);
             tma_load_3d(sOnes, &tmOnes, kv_full, 0, 0, 0);
-            int last_use[C::NST];
+        }
+        const int xchunk = (lane >> 2) & 1;   // chunk of rows lane + 32k holding the term
+        for (int b = 0; b < 2 * C::NST; ++b) {
+            uint8_t *blk = (b < C::NST ? sQB : sDB) + (b % C::NST) * C::XB_BYTES;
 #pragma unroll
-            for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
-            for (int it = 0; it < n_it; ++it) {
-                const int s = it % C::NST, u = it / C::NST;
-                const int h = kvh * G + it % G;
-                const int qt = qt0 + it / G;
-                if (u > 0 && !mbar_wait(&qdo_empty[s], (u - 1) & 1, wc)) break;
-                mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES + 2 * C::XB_BYTES);
+            for (int k = 0; k < kTileM / 32; ++k)
+                reinterpret_cast<uint4 *>(blk + (lane + 32 * k) * kXStepBytes)[xchunk ^ 1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        int last_use[C::NST];
+#pragma unroll
+        for (int s = 0; s < C::NST; ++s) last_use[s] = -1;
+        // the terms of iteration it, loaded one iteration ahead (while the stage is still busy)
+        uint32_t qv[kTileM / 32], dv[kTileM / 32];
+        auto load_terms = [&](int it) {
+            const int h = kvh * G + it % G;
+            const int64_t xo = static_cast<int64_t>(h) * p.Npad + static_cast<int64_t>(qt0 + it / G) * kTileM + lane;
+#pragma unroll
+            for (int k = 0; k < kTileM / 32; ++k) {
+                qv[k] = p.qx[xo + 32 * k];
+                dv[k] = p.dx[xo + 32 * k];
+            }
+        };
+        if (n_it > 0) load_terms(0);
+        for (int it = 0; it < n_it; ++it) {
+            const int s = it % C::NST, u = it / C::NST;
+            const int h = kvh * G + it % G;
+            const int qt = qt0 + it / G;
+            if (u > 0 && !mbar_wait_warp(&qdo_empty[s], (u - 1) & 1, wc)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&qdo_full[s], 2 * C::TILE_BYTES);
                 tma_tile<D>(&tmQ, sQ + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
                 tma_tile<D>(&tmDO, sDO + s * C::TILE_BYTES, &qdo_full[s], p.q_head0 + h, qt * kTileM);
-                tma_load_3d(sQB + s * C::XB_BYTES, &tmQB, &qdo_full[s], 0, h, qt * kTileM);
-                tma_load_3d(sDB + s * C::XB_BYTES, &tmDB, &qdo_full[s], 0, h, qt * kTileM);
-                last_use[s] = u;
             }
+            uint8_t *qb = sQB + s * C::XB_BYTES, *db = sDB + s * C::XB_BYTES;
+#pragma unroll
+            for (int k = 0; k < kTileM / 32; ++k) {
+                const int r = lane + 32 * k;
+                reinterpret_cast<uint4 *>(qb + r * kXStepBytes)[xchunk] = make_uint4(qv[k], 0u, 0u, 0u);
+                reinterpret_cast<uint4 *>(db + r * kXStepBytes)[xchunk] = make_uint4(dv[k], 0u, 0u, 0u);
+            }
+            fence_async_smem();   // visible to the tensor core's operand reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qdo_full[s]);
+            last_use[s] = u;
+            if (it + 1 < n_it) load_terms(it + 1);
+        }
+        if (lane == 0) {
             WaitCtx drain{p.wait_limit_ns, p.status, false};
             mbar_wait(kv_full, 0, drain);
             for (int s = 0; s < C::NST; ++s)
@@ -762,12 +794,9 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
         !encode_tmap_3d(&tk, a.k, D, a.Hkv_total, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW) ||
         !encode_tmap_3d(&tv, a.v, D, a.Hkv_total, a.N, int64_t(D) * 2, ks, C::AW, kTileN, C::SW))
         return cudaErrorInvalidValue;
-    // the dK/dV kernel's extra K-step operands: rows [Npad][Hl][16] bf16, and the block of ones
-    alignas(64) CUtensorMap tqb, tdb, tones;
-    const int64_t xs = int64_t(a.Hl) * kXStepBytes;
-    if (!encode_tmap_3d(&tqb, a.ws + a.L.qb, 16, a.Hl, Npad, kXStepBytes, xs, 16, kTileM, kXStepBytes) ||
-        !encode_tmap_3d(&tdb, a.ws + a.L.db, 16, a.Hl, Npad, kXStepBytes, xs, 16, kTileM, kXStepBytes) ||
-        !encode_tmap_3d(&tones, a.ws + a.L.ones, 16, 1, kTileM, kXStepBytes, kXStepBytes, 16, kTileM, kXStepBytes))
+    // the dK/dV kernel's block of ones for its extra K step (128 rows x 16 bf16)
+    alignas(64) CUtensorMap tones;
+    if (!encode_tmap_3d(&tones, a.ws + a.L.ones, 16, 1, kTileM, kXStepBytes, kXStepBytes, 16, kTileM, kXStepBytes))
         return cudaErrorInvalidValue;
     BwdParams p;
     p.doc_start = reinterpret_cast<const int32_t *>(a.ws + a.L.doc_start);
@@ -779,6 +808,8 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     float *lse2 = reinterpret_cast<float *>(a.ws + a.L.lse2);
     p.delta = delta;
     p.lse2 = lse2;
+    p.qx = reinterpret_cast<const uint32_t *>(a.ws + a.L.qb);
+    p.dx = reinterpret_cast<const uint32_t *>(a.ws + a.L.db);
     p.dq = static_cast<__nv_bfloat16 *>(a.dq);
     p.dk = static_cast<__nv_bfloat16 *>(a.dk);
     p.dv = static_cast<__nv_bfloat16 *>(a.dv);
@@ -799,7 +830,7 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     const int64_t prep_threads = int64_t(a.Hl) * Npad * 32;
     bwd_prep_kernel<D><<<static_cast<unsigned>(ceil_div(prep_threads, 256)), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, delta, lse2,
-        reinterpret_cast<uint4 *>(a.ws + a.L.qb), reinterpret_cast<uint4 *>(a.ws + a.L.db),
+        reinterpret_cast<uint32_t *>(a.ws + a.L.qb), reinterpret_cast<uint32_t *>(a.ws + a.L.db),
         reinterpret_cast<uint4 *>(a.ws + a.L.ones), 1.f / a.scale, p.N, Npad, a.Hl, a.Hq_total, a.q_head0);
     static bool kv_attr[64] = {}, q_attr[64] = {};
     cudaError_t e = set_smem(attn_bwd_dkdv_kernel<D>, C::KV_SMEM, kv_attr);
@@ -807,7 +838,7 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     e = set_smem(attn_bwd_dq_kernel<D>, C::Q_SMEM, q_attr);
     if (e != cudaSuccess) return e;
     attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(int64_t(T) * a.Hkvl), kBwdThreads, C::KV_SMEM, stream>>>(
-        tq, tk, tv, tdo, tqb, tdb, tones, p);
+        tq, tk, tv, tdo, tones, p);
     attn_bwd_dq_kernel<D><<<static_cast<unsigned>(int64_t(T) * a.Hl), kBwdThreads, C::Q_SMEM, stream>>>(
         tq, tk, tv, tdo, p);
     return cudaGetLastError();

@@ -61,8 +61,8 @@ inline WsLayout ws_layout(int64_t N, int Hl, bool backward)
         L.kv_order = off; off += align256(static_cast<size_t>(T) * 4);
         L.delta = off;    off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
         L.lse2 = off;     off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
-        L.qb = off;       off += align256(static_cast<size_t>(T) * kTileM * Hl * kXStepBytes);
-        L.db = off;       off += align256(static_cast<size_t>(T) * kTileM * Hl * kXStepBytes);
+        L.qb = off;       off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
+        L.db = off;       off += align256(static_cast<size_t>(T) * kTileM * Hl * 4);
         L.ones = off;     off += align256(static_cast<size_t>(kTileM) * kXStepBytes);
     } else {
         L.kv_qend = L.kv_order = L.delta = L.lse2 = L.qb = L.db = L.ones = 0;
