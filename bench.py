@@ -44,9 +44,10 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
 
 
 def fwd_launches(n):
-    """Kernels of one forward call over n tokens: the document scan, its carry
-    prefix (only past 2^20 tokens), the fix-up, the work order, the attention."""
-    return 4 + (n > 1 << 20)
+    """Kernels of one forward call over n tokens: the document scan, the fix-up
+    with the work order (one launch up to 2^20 tokens; past that a carry
+    prefix, the fix-up and the order), the attention."""
+    return 3 if n <= 1 << 20 else 5
 
 
 def bwd_launches(n):
