@@ -680,8 +680,11 @@ def run_e2e_pipelined(U, w, inp, args, dev):
     d2h = ho.numel() * 2 + hlse.numel() * 4
     ev_in = [torch.cuda.Event() for _ in range(P)]
     ev_cmp = [torch.cuda.Event() for _ in range(P)]
-    ev_done = torch.cuda.Event()
-    ev_done.record(s_out)
+    ev_out = [torch.cuda.Event() for _ in range(P)]   # rank r's results read back
+    ev_cdone = torch.cuda.Event()                     # a step's attention has read its inputs
+    for e in ev_out:
+        e.record(s_out)
+    ev_cdone.record(s_cmp)
     H2D, D2H = cudart.cudaMemcpyKind.cudaMemcpyHostToDevice, cudart.cudaMemcpyKind.cudaMemcpyDeviceToHost
 
     def copy2d(dst, src, kind, stream, pitch=None, width=None):
@@ -692,7 +695,11 @@ def run_e2e_pipelined(U, w, inp, args, dev):
             raise RuntimeError(f"cudaMemcpy2DAsync: {err}")
 
     def step():
-        s_in.wait_event(ev_done)                  # the previous step has read everything back
+        # Consecutive steps overlap: a step's inputs may land once the previous
+        # step's attention has read its own (its results may still be going back),
+        # and rank r's attention waits only for the previous step's rank r results
+        # to have been read back from the output buffers it rewrites.
+        s_in.wait_event(ev_cdone)
         with torch.cuda.stream(s_in):
             gpos.copy_(hpos, non_blocking=True)
             for r in range(P):
@@ -704,14 +711,16 @@ def run_e2e_pipelined(U, w, inp, args, dev):
         with torch.cuda.stream(s_cmp):
             for r in range(P):
                 s_cmp.wait_event(ev_in[r])
+                s_cmp.wait_event(ev_out[r])
                 U.attn_fwd_fused(gq, gk, gv, gpos, P, r, out=o_seq, lse=lse_all[r * Hl:(r + 1) * Hl], ws=ws)
                 ev_cmp[r].record(s_cmp)
+            ev_cdone.record(s_cmp)
         with torch.cuda.stream(s_out):
             for r in range(P):
                 s_out.wait_event(ev_cmp[r])
                 copy2d(ho.data_ptr() + r * cols, o_seq.data_ptr() + r * cols, D2H, s_out)
                 hlse[r * Hl:(r + 1) * Hl].copy_(lse_all[r * Hl:(r + 1) * Hl], non_blocking=True)
-            ev_done.record(s_out)
+                ev_out[r].record(s_out)
 
     for _ in range(2):
         step()
@@ -731,7 +740,7 @@ def run_e2e_pipelined(U, w, inp, args, dev):
             "steps": args.e2e_steps,
             "path": "pinned host -> device copies (ids, then each rank's K, V and query heads as pitched copies), "
                     "attn_fwd_fused per rank as its heads arrive, each rank's O columns and LSE back on a third "
-                    "stream"}
+                    "stream; a step's input copies start once the previous step's attention has read its inputs"}
 
 
 def run_e2e(U, w, inp, args, dev):
@@ -743,7 +752,8 @@ def run_e2e(U, w, inp, args, dev):
     heads straight from the sequence layout) starts as soon as its heads have
     arrived, and its O columns and LSE rows go back to the host on a third
     stream while the later ranks still compute, so the two copy directions
-    overlap each other and the compute. A workload with a backward copies in
+    overlap each other and the compute (also across steps: the next step's
+    inputs start as soon as this step's attention has read its own). A workload with a backward copies in
     everything, runs the step, and copies the results out."""
     if not w.backward:
         return run_e2e_pipelined(U, w, inp, args, dev)
