@@ -23,7 +23,7 @@ namespace uly {
 namespace {
 
 constexpr int kRelayoutThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;   // vectors in flight per thread (8 measured 2.7 % faster than 4 on llama8b's exchanges)
 
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 {
