@@ -41,9 +41,9 @@
 // The softmax reads its S row, masks only diagonal / document-boundary tiles,
 // keeps a running max with lazy rescaling (O and l are rescaled only when the
 // max grows by more than 2^8), and writes P = exp2(...) back as bf16. The
-// row arithmetic uses the packed fp32x2 FMA / add and the 3-input max; 2/8
-// of the exponentials are evaluated on the FMA pipe (ex2_poly2) so that the
-// special-function unit is not the limit.
+// row arithmetic uses the packed fp32x2 FMA / add and the 3-input max; a
+// quarter of the exponentials (every fourth column pair) are evaluated on the
+// FMA pipe (ex2_poly2) so that the special-function unit is not the limit.
 // Key tiles outside [doc_start(first row), last row] of a tile are never
 // visited by that tile.
 #include "ptx.cuh"
@@ -61,12 +61,13 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10;
 constexpr uint32_t kTmemCols = 512;
-// Column pairs (out of every 8) whose exponentials run on the FMA pipe: the
-// SFU needs 8 cycles per warp instruction, so with only SFU exponentials a
-// 128-column row costs 1024 SFU cycles per warp against ~400 issue slots of
+// One column pair in every kEmuEvery has its exponentials on the FMA pipe:
+// the SFU needs 8 cycles per warp instruction, so with only SFU exponentials
+// a 128-column row costs 1024 SFU cycles per warp against ~400 issue slots of
 // other work; moving part of them to packed polynomials balances the two
-// (2 of 8 measured fastest: 2% over 3 of 8, 6% over 4 of 8).
-constexpr int kEmuPairs = 2;
+// (a quarter measured fastest: 2 % over 3 of 8, 6 % over 4 of 8; spreading
+// them one pair in four rather than two adjacent pairs in eight, 0.6-1.3 %).
+constexpr int kEmuEvery = 4;
 // Register split: launched at 168 per thread (384 x 168 = 64512); the two
 // softmax warpgroups take 216, the producer / MMA warpgroup keeps 72:
 // 256 x 216 + 128 x 72 = 64512.
@@ -651,9 +652,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int e = 0; e < 64; ++e) {
                     float x0, x1;
                     fma2_bcast(x0, x1, s[2 * e], s[2 * e + 1], sl2, -moff);
-                    // kEmuPairs column pairs in 8 take the FMA-pipe exponential, the rest the SFU
+                    // one column pair in kEmuEvery takes the FMA-pipe exponential, the rest the SFU
                     float e0, e1;
-                    if ((e & 7) < kEmuPairs) {
+                    if (e % kEmuEvery == 0) {
                         ex2_poly2(e0, e1, x0, x1);
                     } else {
                         e0 = ex2_approx(x0);
