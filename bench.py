@@ -179,21 +179,29 @@ def workload_work(w, lengths):
 # --------------------------------------------------------------------------- GPU arm
 
 class Timer:
-    """CUDA events around one kind of launch, on the launching stream."""
+    """CUDA events around one kind of launch, on the launching (current)
+    stream. With `external` the events are recorded as nodes of a CUDA graph
+    being captured, and read after its replays (the last replay's times)."""
 
     def __init__(self, stream, enabled: bool):
         self.stream = stream
         self.enabled = enabled
+        self.external = False
         self.ev = {"attn_fwd": [], "attn_bwd": [], "relayout": [], "exchange": [], "merge": []}
+
+    def reset(self):
+        for k in self.ev:
+            self.ev[k] = []
 
     def __call__(self, kind, fn):
         if not self.enabled:
             return fn()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(self.stream)
+        a = torch.cuda.Event(enable_timing=True, external=self.external)
+        b = torch.cuda.Event(enable_timing=True, external=self.external)
+        s = torch.cuda.current_stream()
+        a.record(s)
         r = fn()
-        b.record(self.stream)
+        b.record(s)
         self.ev[kind].append((a, b))
         return r
 
@@ -398,6 +406,23 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     torch.cuda.synchronize()
     U.sync_status(ws)        # raises if a bounded device wait ran out
     timed.enabled = args.kernel_events
+    # One GPU: the step is captured once as a CUDA graph (its launches, with
+    # the per-kind timing events as graph nodes) and replayed; the launch
+    # overhead between the step's kernels then stays off the GPU's timeline.
+    graph = None
+    if world == 1 and args.graph:
+        timed.external = True
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        timed.external = False
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        U.sync_status(ws)
+        run_step = graph.replay
+    else:
+        run_step = step
 
     sampler = ClockSampler(int(str(dev).split(":")[-1]) if ":" in str(dev) else 0)
     sampler.start()
@@ -409,12 +434,13 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(steps):
-        step()
+        run_step()
     t1.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clocks = sampler.stop()
+    ev_steps = 1 if graph is not None else steps   # steps the per-kind events cover
     U.sync_status(ws)
     ms_total = t0.elapsed_time(t1)
     if dist is not None:
@@ -437,14 +463,14 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     long_step = ms_step > 500.0
     bf16_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
     peak_source = "%s %s" % (peak_kind, "sustained" if long_step else "burst")
-    n_fwd = len(timed.ev["attn_fwd"]) // steps if timed.ev["attn_fwd"] else 1   # attention launches per step
-    n_bwd = len(timed.ev["attn_bwd"]) // steps if timed.ev["attn_bwd"] else 1
+    n_fwd = len(timed.ev["attn_fwd"]) // ev_steps if timed.ev["attn_fwd"] else 1   # attention launches per step
+    n_bwd = len(timed.ev["attn_bwd"]) // ev_steps if timed.ev["attn_bwd"] else 1
     fwd_flop_launch = fwd_flop_step / n_fwd
     bwd_flop_launch = bwd_flop_step / n_bwd
     # the attention work of a step over the time its launches took (launches of
     # equal size for Ulysses; the hybrid's ring steps differ in size)
-    achieved = fwd_flop_step / (fwd_sum / steps * 1e-3) / 1e12 if fwd_sum else None
-    bwd_ach = bwd_flop_step / (bwd_sum / steps * 1e-3) / 1e12 if bwd_sum else None
+    achieved = fwd_flop_step / (fwd_sum / ev_steps * 1e-3) / 1e12 if fwd_sum else None
+    bwd_ach = bwd_flop_step / (bwd_sum / ev_steps * 1e-3) / 1e12 if bwd_sum else None
     traffic = lookup_traffic("attn_fwd_kernel", w.name) if world == 1 else None
 
     def roof(kernel, ach, flop_launch, traffic_b):
@@ -493,6 +519,8 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
         "attn_bwd_ms_per_launch": round(bwd_avg, 4) if bwd_avg else None,
         "attn_bwd_tflops": round(bwd_ach, 2) if bwd_ach else None,
         "gpu_launches": launches_per_step * steps,
+        "timing": ("the step captured once as a CUDA graph and replayed; per-kind kernel times from the "
+                   "last replay's event nodes") if graph is not None else "eager launches",
         "clocks": clocks,
     }
     if bwd_avg:
@@ -500,15 +528,15 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
                                    bwd_flop_launch, lookup_traffic("attn_bwd_dkdv_kernel", w.name))
     if rel_sum:
         rbytes = relayout_bytes
-        rb = rbytes / (rel_sum / steps * 1e-3) / 1e9
-        out["relayout"] = {"bytes_per_step": rbytes, "ms_per_step": round(rel_sum / steps, 4),
+        rb = rbytes / (rel_sum / ev_steps * 1e-3) / 1e9
+        out["relayout"] = {"bytes_per_step": rbytes, "ms_per_step": round(rel_sum / ev_steps, 4),
                            "achieved_gbs": round(rb, 1), "peak_gbs": peaks["hbm_gbs"],
                            "peak_source": peak_kind, "frac": round(rb / peaks["hbm_gbs"], 4),
                            "frac_of_spec_8000": round(rb / SPEC_HBM_GBS, 4)}
     if exch_sum:
-        out["exchange_ms_per_step"] = round(exch_sum / steps, 4)
+        out["exchange_ms_per_step"] = round(exch_sum / ev_steps, 4)
     if merge_sum:
-        out["merge_ms_per_step"] = round(merge_sum / steps, 4)
+        out["merge_ms_per_step"] = round(merge_sum / ev_steps, 4)
     if world > 1:
         # device memory one step allocates beyond what is resident before it
         # (exchange buffers and head slices; smaller with more head chunks)
@@ -937,6 +965,8 @@ def main():
     ap.add_argument("--no-fused", dest="fused", action="store_false",
                     help="skip the extra timing of the step with the exchanges fused into the attention")
     ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch the step eagerly instead of replaying it as a CUDA graph (one GPU)")
     ap.add_argument("--ref-seconds", type=float, default=4.0,
                     help="host seconds of oracle work per reference-arm step")
     args = ap.parse_args()
