@@ -298,18 +298,28 @@ def build_fused(U, w, inp, dev):
     return step, fwd_launches(w.N) * P + (bwd_launches(w.N) * P if w.backward else 0), ws
 
 
-def time_fused(U, w, inp, dev, steps, total_flop):
-    """The step with the exchanges fused into the attention (see build_fused)."""
+def time_fused(U, w, inp, dev, steps, total_flop, use_graph=True):
+    """The step with the exchanges fused into the attention (see build_fused),
+    replayed as a CUDA graph like the main step (or launched eagerly)."""
     step, launches, ws = build_fused(U, w, inp, dev)
     stream = torch.cuda.current_stream(dev)
     step()
     torch.cuda.synchronize()
     U.sync_status(ws)
+    run_step = step
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        U.sync_status(ws)
+        run_step = graph.replay
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(steps):
-        step()
+        run_step()
     t1.record(stream)
     torch.cuda.synchronize()
     U.sync_status(ws)
@@ -553,7 +563,7 @@ def measure(U, w, dev, args, steps, warmup, world, rank, dist, headline):
     if headline:
         out["e2e"] = run_e2e(U, w, inp, args, dev) if (args.e2e_steps > 0 and world == 1) else None
     if world == 1 and args.fused and not attn_ranks and not w.ulysses:
-        out["fused_step"] = time_fused(U, w, inp, dev, steps, total_flop)
+        out["fused_step"] = time_fused(U, w, inp, dev, steps, total_flop, args.graph)
     if headline and rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, inp, args)
     del inp, step, ws
