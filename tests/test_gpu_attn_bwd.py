@@ -34,6 +34,9 @@ CASES = [
     ([5] * 40, 2, 2, 128),
     ([1000, 24], 8, 2, 128),
     ([513, 511], 2, 2, 32),
+    ([600, 700, 29], 6, 2, 64),         # odd group size: three query heads per KV head
+    ([1100, 3], 3, 1, 128),
+    ([900, 100, 44], 8, 1, 64),         # group of 8: one dK/dV CTA sums eight heads
 ]
 
 
