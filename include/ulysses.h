@@ -286,9 +286,11 @@ void ulysses_set_wait_limit_ns(int64_t ns);
 /*
  * Test hook for the failure path (no counterpart in the pages). Bit 0: later
  * forward launches make their first CTA wait on a barrier that nothing ever
- * arrives on; the bounded wait runs out, the launch drains and returns, and
- * ulysses_sync_status() reports ULYSSES_ERR_TIMEOUT. Nothing faults or hangs.
- * 0 (the default) disables it.
+ * arrives on; bit 1: the same for the first CTA of the backward's dK/dV
+ * kernel. The bounded wait runs out, the launch drains and returns (the
+ * backward's dQ kernel, launched after it, finds the status set and skips its
+ * work), and ulysses_sync_status() reports ULYSSES_ERR_TIMEOUT. Nothing faults
+ * or hangs. 0 (the default) disables it.
  */
 void ulysses_set_debug_flags(uint32_t flags);
 

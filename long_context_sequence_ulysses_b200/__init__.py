@@ -484,7 +484,8 @@ def set_wait_limit_ns(ns: int) -> None:
 
 
 def set_debug_flags(flags: int) -> None:
-    """Test hook: bit 0 makes later forward launches run one bounded wait out."""
+    """Test hook: bit 0 makes later forward launches, bit 1 later backward
+    launches, run one bounded wait out."""
     _lib.ulysses_set_debug_flags(int(flags))
 
 

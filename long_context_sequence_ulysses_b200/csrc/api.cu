@@ -351,6 +351,7 @@ static int attn_bwd_common(const char *name, const void *q, const void *k, const
     a.ws = static_cast<char *>(ws);
     a.L = L;
     a.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
+    a.debug_flags = g_debug_flags;
     e = launch_attn_bwd(a, s);
     if (e == cudaErrorNotSupported) return fail(ULYSSES_ERR_UNSUPPORTED, "%s: not built", name);
     if (e != cudaSuccess) return cuda_fail(e, name);

@@ -82,6 +82,7 @@ struct BwdParams {
     float scale_log2, scale;
     uint32_t *status;
     uint64_t wait_limit_ns;
+    uint32_t debug_flags;   // bit 1: the first dK/dV CTA's element-wise warps wait on a barrier nobody arrives on
 };
 
 template <int D>
@@ -254,7 +255,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *p_ready = dp_full + 1;          // P^T(i) stored (all compute threads)
     uint64_t *acc_done = p_ready + 1;
     uint64_t *mma_done = acc_done + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *never = mma_done + 1;           // never arrived on (timeout test only)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(never + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int item = blockIdx.x;
@@ -277,6 +279,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(p_ready, kParts * 128);
         mbar_init(acc_done, 1);
         mbar_init(mma_done, 1);
+        mbar_init(never, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -435,7 +438,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float sl2 = p.scale_log2;
         const uint32_t col = static_cast<uint32_t>(part * kPartCols);   // this part's columns in S^T / dP^T
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
+        if ((p.debug_flags & 2u) && blockIdx.x == 0) ok = mbar_wait_warp(never, 0, wc);   // runs out
+        for (int it = 0; ok && it < n_it; ++it) {
             const int q0 = (qt0 + it / G) * kTileM + part * kPartCols;   // first query of this part
             // warp-uniform wait: the tcgen05.ld below needs the whole warp converged
             if (!mbar_wait_warp(s_full, it & 1, wc)) { ok = false; break; }
@@ -826,6 +830,7 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     p.scale_log2 = a.scale * kLog2e;
     p.status = reinterpret_cast<uint32_t *>(a.ws + a.L.status);
     p.wait_limit_ns = a.wait_limit_ns;
+    p.debug_flags = a.debug_flags;
 
     const int64_t prep_threads = int64_t(a.Hl) * Npad * 32;
     bwd_prep_kernel<D><<<static_cast<unsigned>(ceil_div(prep_threads, 256)), 256, 0, stream>>>(

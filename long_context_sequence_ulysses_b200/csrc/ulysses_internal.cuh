@@ -134,6 +134,7 @@ struct BwdLaunch {
     char *ws;
     WsLayout L;
     uint64_t wait_limit_ns;
+    uint32_t debug_flags = 0;
 };
 cudaError_t launch_attn_bwd(const BwdLaunch &a, cudaStream_t stream);
 
