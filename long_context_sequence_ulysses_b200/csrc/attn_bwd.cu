@@ -149,7 +149,8 @@ __device__ __forceinline__ uint32_t bf16_hi_lo(float v)
     return pack_bf16x2(__bfloat162float(hi), rest);
 }
 
-// D_i = sum_c dO_ic O_ic and -LSE_i * log2(e), one warp per (head, padded row).
+// D_i = sum_c dO_ic O_ic and -LSE_i * log2(e), D/8 lanes per (head, padded
+// row): each lane one 16-byte chunk of O and dO, so a warp takes 32/(D/8) rows.
 // For the dK/dV kernel the same two terms also go, as hi/lo bf16 pairs, into
 // an extra K step of its products: qx[h][i] holds -LSE_i / scale (S^T + that,
 // times scale*log2(e), is the exponent of P^T), dx[h][i] holds -D_i (dP^T +
@@ -169,21 +170,24 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
         ones[2 * threadIdx.x] = make_uint4(one2, 0u, 0u, 0u);
         ones[2 * threadIdx.x + 1] = make_uint4(0u, 0u, 0u, 0u);
     }
-    const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    constexpr int kLanesPerRow = D / 8;
+    static_assert(kLanesPerRow >= 1 && kLanesPerRow <= 32 && 32 % kLanesPerRow == 0, "lanes per row");
     const int lane = threadIdx.x & 31;
-    if (w >= static_cast<int64_t>(Hl) * Npad) return;
-    const int h = static_cast<int>(w / Npad);
-    const int i = static_cast<int>(w % Npad);
+    const int64_t w = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * (32 / kLanesPerRow) +
+                      lane / kLanesPerRow;
+    const int sl = lane % kLanesPerRow;
+    const bool in_range = w < static_cast<int64_t>(Hl) * Npad;
+    const int h = in_range ? static_cast<int>(w / Npad) : 0;
+    const int i = in_range ? static_cast<int>(w % Npad) : N;
     float acc = 0.f;
     if (i < N) {
         const int64_t off = (static_cast<int64_t>(i) * Hq_total + q_head0 + h) * D;
-        const uint4 *po = reinterpret_cast<const uint4 *>(o + off);
-        const uint4 *pd = reinterpret_cast<const uint4 *>(dout + off);
-        for (int v = lane; v < D / 8; v += 32) acc += dot8_bf16(po[v], pd[v]);
+        acc = dot8_bf16(reinterpret_cast<const uint4 *>(o + off)[sl], reinterpret_cast<const uint4 *>(dout + off)[sl]);
     }
+    // the row's lanes in a fixed tree (every lane of the warp takes part)
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (in_range && sl == 0) {
         const float lse_i = i < N ? lse[static_cast<int64_t>(h) * N + i] : CUDART_INF_F;
         delta[w] = i < N ? acc : 0.f;
         lse2[w] = i < N ? -lse_i * kLog2e : -CUDART_INF_F;
@@ -832,7 +836,7 @@ cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream)
     p.wait_limit_ns = a.wait_limit_ns;
     p.debug_flags = a.debug_flags;
 
-    const int64_t prep_threads = int64_t(a.Hl) * Npad * 32;
+    const int64_t prep_threads = int64_t(a.Hl) * Npad * (D / 8);   // D/8 lanes per (head, row)
     bwd_prep_kernel<D><<<static_cast<unsigned>(ceil_div(prep_threads, 256)), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, delta, lse2,
         reinterpret_cast<uint32_t *>(a.ws + a.L.qb), reinterpret_cast<uint32_t *>(a.ws + a.L.db),
