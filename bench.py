@@ -910,7 +910,8 @@ def _oracle_step(w, inp, sl, rate, seconds_target, seed):
 def cpu_baseline(w, inp, args, seconds_target: float = 15.0):
     """The fp64 oracle timed on this host's cores on a bounded sample of rank
     0's rows; its rate is scaled to TFLOP/s with the same FLOP count per pair."""
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    import oracle
+    threads = oracle.max_threads()   # the threads its loops actually use
     sl = _oracle_slice(w, inp)
     dt, pr, nrows = _oracle_step(w, inp, sl, _oracle_rate(w, inp, sl), seconds_target, seed=2)
     flop = 4.0 * w.d * pr
@@ -930,7 +931,11 @@ def run_reference(args):
         return
     w = WORKLOADS["llama8b" if args.workload == "all" else args.workload]
     inp = make_inputs(w, device="cpu")
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    import oracle
+    if world > 1:
+        # the launcher gives every rank one host thread; the other ranks do no work
+        oracle.set_num_threads(os.cpu_count() or 1)
+    threads = oracle.max_threads()
     sl = _oracle_slice(w, inp)
     rate = _oracle_rate(w, inp, sl)
     times, pairs = [], []

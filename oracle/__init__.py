@@ -57,6 +57,10 @@ def _load():
             lib.oracle_head_to_seq.restype = I32
             lib.oracle_doc_start.argtypes = [P, I64, P]
             lib.oracle_doc_start.restype = None
+            lib.oracle_set_num_threads.argtypes = [I32]
+            lib.oracle_set_num_threads.restype = None
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = I32
             lib.oracle_attn_fwd_rows.argtypes = [P, P, P, P, I64, I32, I32, I32, F64, P, I64, P, P]
             lib.oracle_attn_fwd_rows.restype = I32
             lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, I64, I32, I32, I32, F64, P, P, P, P, P]
@@ -273,3 +277,13 @@ def out_proj(o_heads, w_o, rows: Optional[Sequence[int]] = None):
     if rows is not None:
         seq = seq[np.asarray(rows, dtype=np.int64)]
     return seq @ _f64(w_o).T
+
+
+def set_num_threads(n: int) -> None:
+    """Host threads of the oracle's loops (no effect on its arithmetic)."""
+    _load().oracle_set_num_threads(int(n))
+
+
+def max_threads() -> int:
+    """Threads the oracle's loops use."""
+    return int(_load().oracle_max_threads())

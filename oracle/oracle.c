@@ -30,6 +30,7 @@
  * All bf16 inputs arrive as raw 16-bit patterns and are widened exactly.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -526,3 +527,13 @@ void oracle_merge(const double *o_parts, const double *lse_parts, int R, int64_t
             lse[(int64_t)h * M + m] = L;
         }
 }
+
+/* Host threads of the loops above (no arithmetic): a launcher that gives the
+ * process one thread (torchrun does, for each rank) can hand rank 0 the whole
+ * host back. */
+void oracle_set_num_threads(int n)
+{
+    if (n > 0) omp_set_num_threads(n);
+}
+
+int oracle_max_threads(void) { return omp_get_max_threads(); }

@@ -532,3 +532,19 @@ def test_projections_against_torch_matmul():
     wo = _bf((hidden, H * d), 10)
     seq = o.double().permute(1, 0, 2, 3).reshape(N, H * d)
     np.testing.assert_allclose(oracle.out_proj(o, wo), (seq @ wo.double().T).numpy(), rtol=0, atol=1e-12)
+
+
+def test_thread_count_setting_leaves_results_unchanged():
+    """The host thread count of the oracle's loops is a launch setting: the
+    same inputs give bit-identical results with one thread and with all."""
+    n0 = oracle.max_threads()
+    c = random_case(300, 2, 1, 32, [200, 100], seed=5, device="cpu")
+    try:
+        oracle.set_num_threads(1)
+        assert oracle.max_threads() == 1
+        o1, l1 = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    finally:
+        oracle.set_num_threads(n0)
+    assert oracle.max_threads() == n0
+    o2, l2 = oracle.attn_fwd(c["q"], c["k"], c["v"], c["position_ids"])
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
