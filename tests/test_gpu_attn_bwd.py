@@ -243,3 +243,42 @@ def test_bwd_fused_equals_slice():
         assert torch.equal(dq_f[:, qs], dq)
         assert torch.equal(dk_f[:, ks], dk)
         assert torch.equal(dv_f[:, ks], dv)
+
+
+@pytest.mark.parametrize("P,H,Hkv,d,lengths", [
+    (2, 6, 2, 64, [600, 700, 30]),      # group of 3: the forward pairs consecutive query tiles
+    (4, 8, 4, 32, [500, 300, 200, 24]),
+    (2, 4, 2, 128, [1000, 24]),
+])
+def test_fused_small_shapes_against_oracle(P, H, Hkv, d, lengths):
+    """The fused forward and backward of every rank on small sequence-sharded
+    buffers, every element of every rank's heads against the oracle on that
+    rank's head slice (the fused path at group sizes and head dimensions the
+    workload tests do not reach)."""
+    import long_context_sequence_ulysses_b200 as U
+    N = sum(lengths)
+    c = random_case(N, H, Hkv, d, lengths, seed=N + H + d, device="cuda", with_grad_out=True)
+    pos = c["position_ids"]
+    Hl, Hkvl = H // P, Hkv // P
+    nan = float("nan")
+    o_seq = torch.full_like(c["q"], nan)
+    dq_s, dk_s, dv_s = (torch.full_like(c[x], nan) for x in ("q", "k", "v"))
+    lse_all = torch.empty((H, N), dtype=torch.float32, device="cuda")
+    for r in range(P):
+        U.attn_fwd_fused(c["q"], c["k"], c["v"], pos, P, r, out=o_seq, lse=lse_all[r * Hl:(r + 1) * Hl])
+    for r in range(P):
+        U.attn_bwd_fused(c["q"], c["k"], c["v"], o_seq, c["do"], lse_all[r * Hl:(r + 1) * Hl], pos, P, r,
+                         dq=dq_s, dk=dk_s, dv=dv_s)
+    torch.cuda.synchronize()
+    for x in (o_seq, dq_s, dk_s, dv_s):
+        assert not torch.isnan(x.float()).any()          # the ranks together wrote every head
+    cpu = {x: c[x].cpu() for x in ("q", "k", "v", "do")}
+    for r in range(P):
+        qs, ks = slice(r * Hl, (r + 1) * Hl), slice(r * Hkvl, (r + 1) * Hkvl)
+        rq, rk, rv, ro, rl = oracle.attn_bwd(cpu["q"][:, qs].contiguous(), cpu["k"][:, ks].contiguous(),
+                                             cpu["v"][:, ks].contiguous(), cpu["do"][:, qs].contiguous(), pos.cpu())
+        assert_close(f"O rank {r}", bf16_to_f64(o_seq[:, qs]), ro)
+        assert_close(f"LSE rank {r}", lse_all[qs].double().cpu().numpy(), rl)
+        assert_grad_close(f"dQ rank {r}", bf16_to_f64(dq_s[:, qs]), rq)
+        assert_grad_close(f"dK rank {r}", bf16_to_f64(dk_s[:, ks]), rk)
+        assert_grad_close(f"dV rank {r}", bf16_to_f64(dv_s[:, ks]), rv)
